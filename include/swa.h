@@ -1,0 +1,195 @@
+/*
+ * swa.h -- C ABI of the B200 (sm_100a) causal sliding-window attention library.
+ *
+ * The operation (M003 note "weight sparsity vs attention sparsity", section 03;
+ * Chapter 10 "local and sparse attention: SWA and DSA", section 10.1):
+ *
+ *   a query at logical position i may read the key at logical position j iff
+ *   max(0, i - W + 1) <= j <= i   (the window of W keys includes the query's
+ *   own position); scores are scale * <q_i, k_j> on those pairs only, the
+ *   softmax is normalised over those pairs only, and the output is the
+ *   softmax-weighted sum of the matching value rows.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major (C order), bfloat16 unless stated.  Query
+ *    tensors are [B, H, rows, d]; key/value tensors are [B, Hkv, rows, d].
+ *    Query head h reads key/value head h / (H / Hkv) (contiguous groups of
+ *    G = H / Hkv query heads share one key/value head).
+ *  - Every pointer argument named as device memory must point to memory of
+ *    the current CUDA device, 16-byte aligned.  The caller owns all memory;
+ *    the library never allocates, frees or retains a pointer after a call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every compute call only validates its arguments on the host
+ *    and enqueues kernels on `stream`; it returns before the work finishes.
+ *  - d (head dim) must be 64 or 128.  W >= 1; W >= the sequence length means
+ *    plain causal attention.  `scale` must be finite and > 0.
+ *  - Return value: SWA_OK or one of the error codes below.  Nothing is
+ *    printed and no exception crosses the ABI.  Arguments are checked before
+ *    anything is enqueued: an invalid argument enqueues nothing.  Errors found
+ *    on the device (a negative position, a wait that timed out) set a device
+ *    status word that swa_get_device_status() reads and clears.
+ *  - Thread safety: calls are stateless apart from a per-process cache of a
+ *    driver entry point, which is set up once under a lock.
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SWA_API __attribute__((visibility("default")))
+#else
+#define SWA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SWA_OK 0
+#define SWA_ERR_INVALID_ARG 1 /* a size, pointer, alignment or value is out of range   */
+#define SWA_ERR_UNSUPPORTED 2 /* valid request outside what the kernels implement      */
+#define SWA_ERR_CUDA 3        /* a CUDA runtime or driver call failed                  */
+#define SWA_ERR_WORKSPACE 4   /* workspace missing or smaller than required            */
+#define SWA_ERR_TIMEOUT 5     /* a device-side wait gave up (reported by get_status)   */
+#define SWA_ERR_DEVICE 6      /* a device-side argument check failed (get_status)      */
+
+/* Human-readable name of a status code (static string, never NULL). */
+SWA_API const char *swa_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+SWA_API int swa_version(void);
+
+/*
+ * swa_block_meta -- tile metadata built on the device.
+ * Passage: M003 note section 04 (tiles that are entirely invisible are
+ * skipped, entirely visible tiles need no mask, partially visible tiles are
+ * computed whole and masked at the boundary) and section 07 (metadata is
+ * built for the pattern and timed with the kernel).
+ *
+ * key_mode 0 (linear): query row i of sequence b sits at logical position
+ *   q_pos0[b] + i (q_pos0 == NULL: 0), 0 <= i < n_q; key column j sits at
+ *   position j, 0 <= j < n_k.
+ * key_mode 1 (ring + chunk, Chapter 10 section 10.2): queries are a chunk at
+ *   positions q_pos0[b] + i (q_pos0 is the chunk start, required); the key
+ *   axis is the W slots of a ring buffer in physical order (slot s holds the
+ *   most recent position p < q_pos0[b] with p mod W == s, or nothing), tiled
+ *   on their own, followed by the n_q chunk keys at q_pos0[b] + t, tiled on
+ *   their own.  n_k is ignored.
+ *
+ * Tiles are tile_q x tile_k (each 1..1024); ragged last tiles are clipped to
+ * their in-range coordinates.  Outputs (device memory, caller-allocated):
+ *   classes: int8 [B, nqt, nkt] (may be NULL): 0 skip, 1 full, 2 partial;
+ *   ranges:  int32 [B, nqt, 4]  (may be NULL): {live tiles, full tiles,
+ *            first live tile, last live tile} (-1 when there is none);
+ * with nqt = ceil(n_q / tile_q) and nkt = ceil(n_k / tile_k) (mode 0) or
+ * ceil(W / tile_k) + ceil(n_q / tile_k) (mode 1).
+ */
+SWA_API int swa_block_meta(int key_mode, int B, int64_t n_q, int64_t n_k, const int64_t *q_pos0,
+                   int64_t W, int tile_q, int tile_k, int8_t *classes, int32_t *ranges,
+                   void *stream);
+
+/*
+ * swa_attn_fwd -- tile-skipping prefill forward.
+ * Passage: M003 note sections 03-04; Chapter 10 section 10.1.
+ *   q:   [B, H, N, d]    bf16, device     k, v: [B, Hkv, N, d] bf16, device
+ *   out: [B, H, N, d]    bf16, device (written)
+ *   lse: [B, H, N] fp32, device, or NULL: natural-log log-sum-exp of the
+ *        scaled scores of each row over its allowed keys.
+ * Query and key row i both sit at logical position i.  Only key tiles that
+ * hold an allowed pair are loaded; only partially visible tiles are masked.
+ * Limits: 1 <= N < 2^30, H % Hkv == 0.
+ */
+SWA_API int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                 int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream);
+
+/*
+ * swa_attn_chunk_ring -- chunked prefill over a W-slot ring-buffer KV cache.
+ * Passage: Chapter 10 section 10.2 (a chunk of T_q queries needs the union of
+ * W + T_q - 1 keys; the persistent cache keeps only the last W); M003 note
+ * section 06 (logical positions keep growing while slots are reused);
+ * "Dense attention vs sparse SWA" blog section 3.2 (the circular cache).
+ *   q:            [B, H, Tq, d]    bf16, device   chunk queries
+ *   k_new, v_new: [B, Hkv, Tq, d]  bf16, device   chunk keys / values
+ *   k_ring, v_ring: [B, Hkv, W, d] bf16, device   ring cache; before the call
+ *                 slot s of sequence b holds the most recent position
+ *                 p < q_start[b] with p mod W == s (empty if none)
+ *   q_start: int64 [B], device: logical position of the chunk's first query
+ *                 (>= 0; a negative value sets SWA_ERR_DEVICE on the device)
+ *   out: [B, H, Tq, d] bf16, device;  lse: [B, H, Tq] fp32 or NULL.
+ * Query t sits at q_start[b] + t and attends to ring keys and chunk keys by
+ * logical position.  If update_ring != 0, after the attention (same stream)
+ * the chunk rows whose positions are among the last W are written into slots
+ * position mod W, so the ring then serves the next chunk or decode step.
+ * The ring is only written when update_ring != 0.  Limits: 1 <= Tq < 2^30,
+ * W < 2^29.
+ */
+SWA_API int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,
+                        void *v_ring, const int64_t *q_start, void *out, float *lse, int B,
+                        int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                        int update_ring, void *stream);
+
+/*
+ * swa_ring_write -- append a chunk of keys/values to a ring cache.
+ * Passage: blog section 3.2 (slot = position mod W once the ring is full);
+ * M003 note section 06 (update the position-to-slot map before reuse).
+ * Writes rows t of k_new/v_new [B, Hkv, T, d] whose positions
+ * q_start[b] + t are among the last W (q_start[b] + t >= q_start[b] + T - W)
+ * into slot (q_start[b] + t) mod W of k_ring/v_ring [B, Hkv, W, d].
+ */
+SWA_API int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_ring,
+                   const int64_t *q_start, int B, int Hkv, int64_t T, int d, int64_t W,
+                   void *stream);
+
+/*
+ * swa_decode_workspace_bytes -- bytes of scratch swa_attn_decode_ring needs
+ * for these sizes (split partial results: fp32 O, running max and sum).
+ */
+SWA_API size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int64_t W);
+
+/*
+ * swa_attn_decode_ring -- batched single-token decode from a ring cache.
+ * Passage: blog section 3.2 (circular cache); sparse-attention taxonomy
+ * page section 1 (a decode step is bound by reading the KV cache from HBM).
+ *   q: [B, H, d] bf16, device: the query of sequence b at logical position
+ *      pos[b]; its own key/value are already in slot pos[b] mod W.
+ *   k_ring, v_ring: [B, Hkv, W, d] bf16, device: slot s holds the most
+ *      recent position p <= pos[b] with p mod W == s (empty if none).
+ *   pos: int64 [B], device (>= 0).   out: [B, H, d] bf16, device.
+ *   lse: [B, H] fp32 or NULL.
+ *   workspace: device scratch of at least swa_decode_workspace_bytes(...)
+ *      bytes, caller-owned; contents on entry are ignored.
+ * Each key/value slot is read from HBM once for all G query heads of its
+ * group; the key range is split across CTAs and merged in a second kernel.
+ */
+SWA_API int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
+                         const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
+                         int d, int64_t W, float scale, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * swa_ring_slot_positions -- the logical position held by every ring slot.
+ * Passage: M003 note section 06 (logical vs physical slots); blog section 3.2.
+ * For sequence b after positions 0 .. n_written[b]-1 were written:
+ *   slot_pos[b, s] = the largest p < n_written[b] with p mod W == s, or -1.
+ * n_written: int64 [B] device; slot_pos: int64 [B, W] device (written).
+ */
+SWA_API int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,
+                            void *stream);
+
+/*
+ * swa_get_device_status -- synchronise `stream`, then read and clear the
+ * device status word of the current device: SWA_OK, SWA_ERR_TIMEOUT (a
+ * device-side wait gave up; the kernel returned early and its outputs are
+ * invalid) or SWA_ERR_DEVICE (a device-side argument check failed).
+ * Returns SWA_ERR_CUDA if the synchronisation itself reports an error.
+ */
+SWA_API int swa_get_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

@@ -1,0 +1,190 @@
+"""Causal sliding-window attention for NVIDIA B200 (sm_100a).
+
+A query at logical position i reads the keys at positions
+max(0, i - W + 1) .. i (the window includes the query's own position), and
+the softmax is taken over those pairs only.  Every step runs in the CUDA
+kernels of ``libswa.so`` behind the C ABI of ``include/swa.h``; this module
+only marshals torch tensors (device memory, current stream) into those calls.
+The function names match the C entry points.
+
+Layouts (row-major bf16): queries ``[B, H, rows, d]``, keys/values
+``[B, Hkv, rows, d]``, ring caches ``[B, Hkv, W, d]``; query head h reads
+key/value head ``h // (H // Hkv)``.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from ._native import SwaError, check, lib, status_name  # noqa: F401
+
+__all__ = [
+    "SwaError",
+    "lib",
+    "swa_block_meta",
+    "swa_attn_fwd",
+    "swa_attn_chunk_ring",
+    "swa_ring_write",
+    "swa_decode_workspace_bytes",
+    "swa_attn_decode_ring",
+    "swa_ring_slot_positions",
+    "swa_get_device_status",
+    "swa_version",
+]
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device=None):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t, name, dtype=torch.bfloat16, dims=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dims, got {t.dim()}")
+
+
+def swa_version() -> int:
+    return int(lib().swa_version())
+
+
+def swa_block_meta(key_mode: int, n_q: int, n_k: int, W: int, tile_q: int, tile_k: int,
+                   q_pos0: torch.Tensor | None = None, B: int | None = None,
+                   classes: torch.Tensor | None = None, ranges: torch.Tensor | None = None,
+                   device=None):
+    """Tile classes (int8 [B,nqt,nkt]: 0 skip, 1 full, 2 partial) and ranges (int32 [B,nqt,4])."""
+    if q_pos0 is not None:
+        _need(q_pos0, "q_pos0", torch.int64, 1)
+        B = q_pos0.numel()
+        device = q_pos0.device
+    if B is None:
+        raise ValueError("B is required when q_pos0 is None")
+    device = torch.device("cuda") if device is None else torch.device(device)
+    nqt = (n_q + tile_q - 1) // tile_q
+    nkt = ((n_k + tile_k - 1) // tile_k if key_mode == 0
+           else (W + tile_k - 1) // tile_k + (n_q + tile_k - 1) // tile_k)
+    if classes is None:
+        classes = torch.empty((B, nqt, nkt), dtype=torch.int8, device=device)
+    if ranges is None:
+        ranges = torch.empty((B, nqt, 4), dtype=torch.int32, device=device)
+    check("swa_block_meta", lib().swa_block_meta(key_mode, B, n_q, n_k, _ptr(q_pos0), W, tile_q,
+                                                 tile_k, _ptr(classes), _ptr(ranges),
+                                                 _stream(device)))
+    return classes, ranges
+
+
+def swa_attn_fwd(q, k, v, W: int, scale: float | None = None, out=None, lse=None,
+                 return_lse: bool = False):
+    """Prefill forward: q [B,H,N,d], k/v [B,Hkv,N,d] -> out [B,H,N,d] (and lse [B,H,N])."""
+    _need(q, "q", dims=4)
+    _need(k, "k", dims=4)
+    _need(v, "v", dims=4)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, N, d) or tuple(v.shape) != (B, Hkv, N, d):
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dims=4)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    check("swa_attn_fwd", lib().swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H,
+                                             Hkv, N, d, W, scale, _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_attn_chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, scale: float | None = None,
+                        update_ring: bool = False, out=None, lse=None, return_lse: bool = False):
+    """Chunked prefill on a ring cache: q [B,H,Tq,d], chunk k/v [B,Hkv,Tq,d], ring [B,Hkv,W,d]."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"),
+                 (v_ring, "v_ring")):
+        _need(t, n, dims=4)
+    _need(q_start, "q_start", torch.int64, 1)
+    B, H, Tq, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    check("swa_attn_chunk_ring",
+          lib().swa_attn_chunk_ring(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring),
+                                    _ptr(q_start), _ptr(out), _ptr(lse), B, H, Hkv, Tq, d, W,
+                                    scale, 1 if update_ring else 0, _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_ring_write(k_new, v_new, k_ring, v_ring, q_start):
+    """Write the chunk rows among the last W positions into slot position mod W (in place)."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"), (v_ring, "v_ring")):
+        _need(t, n, dims=4)
+    _need(q_start, "q_start", torch.int64, 1)
+    B, Hkv, T, d = k_new.shape
+    W = k_ring.shape[2]
+    check("swa_ring_write", lib().swa_ring_write(_ptr(k_new), _ptr(v_new), _ptr(k_ring),
+                                                 _ptr(v_ring), _ptr(q_start), B, Hkv, T, d, W,
+                                                 _stream(k_new.device)))
+
+
+def swa_decode_workspace_bytes(B: int, H: int, Hkv: int, d: int, W: int) -> int:
+    return int(lib().swa_decode_workspace_bytes(B, H, Hkv, d, W))
+
+
+def swa_attn_decode_ring(q, k_ring, v_ring, pos, scale: float | None = None, workspace=None,
+                         out=None, lse=None, return_lse: bool = False):
+    """Decode: q [B,H,d] at positions pos [B] over ring caches [B,Hkv,W,d] -> out [B,H,d]."""
+    _need(q, "q", dims=3)
+    _need(k_ring, "k_ring", dims=4)
+    _need(v_ring, "v_ring", dims=4)
+    _need(pos, "pos", torch.int64, 1)
+    B, H, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = swa_decode_workspace_bytes(B, H, Hkv, d, W)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    check("swa_attn_decode_ring",
+          lib().swa_attn_decode_ring(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(pos), _ptr(out),
+                                     _ptr(lse), B, H, Hkv, d, W, scale, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_ring_slot_positions(n_written, W: int, out=None):
+    """int64 [B, W]: the logical position each ring slot holds after n_written[b] writes (-1 empty)."""
+    _need(n_written, "n_written", torch.int64, 1)
+    B = n_written.numel()
+    if out is None:
+        out = torch.empty((B, W), dtype=torch.int64, device=n_written.device)
+    check("swa_ring_slot_positions", lib().swa_ring_slot_positions(
+        B, _ptr(n_written), W, _ptr(out), _stream(n_written.device)))
+    return out
+
+
+def swa_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word as a status code."""
+    s = _stream() if stream is None else stream
+    return int(lib().swa_get_device_status(s))

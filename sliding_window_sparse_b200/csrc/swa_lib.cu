@@ -1,0 +1,329 @@
+// swa_lib.cu -- the C ABI declared in include/swa.h.
+//
+// Host code only validates arguments, encodes TMA tensor maps and enqueues
+// kernels on the caller's stream.  All kernels live in the headers included
+// below, compiled in this single translation unit so they share the one
+// device status word g_swa_status.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/swa.h"
+#include "sm100.cuh"
+#include "swa_decode.cuh"
+#include "swa_fwd.cuh"
+#include "swa_meta.cuh"
+#include "swa_tile.cuh"
+
+namespace {
+
+using swa::kBK;
+using swa::kBQ;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor map over [planes, rows, d] with a 64-column x box_rows box,
+// 128-byte swizzle; rows past `rows` read as zero.
+int make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t planes, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return SWA_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : SWA_ERR_CUDA;
+}
+
+inline int check_launch() {
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+inline bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+int common_checks(int B, int H, int Hkv, int d, int64_t W, float scale) {
+  if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  if (W < 1 || !good_scale(scale)) return SWA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H > (1 << 24)) return SWA_ERR_UNSUPPORTED;
+  return SWA_OK;
+}
+
+template <int D, int MODE>
+int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+               const CUtensorMap &tkr, const CUtensorMap &tvr, const swa::FwdParams &p,
+               cudaStream_t st) {
+  using L = swa::FwdLayout<D>;
+  auto kern = swa::fwd_kernel<D, MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
+      cudaSuccess)
+    return SWA_ERR_CUDA;
+  const int64_t blocks = static_cast<int64_t>(p.nqt) * p.B * p.H;
+  if (blocks > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(blocks), swa::kFwdThreads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr,
+                                                                          p);
+  return check_launch();
+}
+
+// Split policy of the decode path (shared by the workspace query and the launch).
+void decode_split(int B, int Hkv, int64_t W, int *chunk, int *splits) {
+  int c = 512;
+  while (c > 128 && static_cast<int64_t>(B) * Hkv * ((W + c - 1) / c) < 4 * 148) c >>= 1;
+  *chunk = c;
+  *splits = static_cast<int>((W + c - 1) / c);
+}
+
+template <int D, int G>
+int launch_decode(const swa::DecodeParams &p, cudaStream_t st) {
+  dim3 grid(p.splits, p.Hkv, p.B);
+  swa::decode_split_kernel<D, G><<<grid, swa::kDecWarps * 32, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+  swa::decode_combine_kernel<D><<<static_cast<unsigned>(p.B * p.H), D, 0, st>>>(p);
+  return check_launch();
+}
+
+template <int D>
+int dispatch_decode_g(int G, const swa::DecodeParams &p, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode<D, 1>(p, st);
+    case 2: return launch_decode<D, 2>(p, st);
+    case 4: return launch_decode<D, 4>(p, st);
+    case 8: return launch_decode<D, 8>(p, st);
+    default: return SWA_ERR_UNSUPPORTED;
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char *swa_status_string(int status) {
+  switch (status) {
+    case SWA_OK: return "SWA_OK";
+    case SWA_ERR_INVALID_ARG: return "SWA_ERR_INVALID_ARG";
+    case SWA_ERR_UNSUPPORTED: return "SWA_ERR_UNSUPPORTED";
+    case SWA_ERR_CUDA: return "SWA_ERR_CUDA";
+    case SWA_ERR_WORKSPACE: return "SWA_ERR_WORKSPACE";
+    case SWA_ERR_TIMEOUT: return "SWA_ERR_TIMEOUT";
+    case SWA_ERR_DEVICE: return "SWA_ERR_DEVICE";
+    default: return "SWA_ERR_UNKNOWN";
+  }
+}
+
+int swa_version(void) { return (1 << 16) | 0; }
+
+int swa_block_meta(int key_mode, int B, int64_t n_q, int64_t n_k, const int64_t *q_pos0,
+                   int64_t W, int tile_q, int tile_k, int8_t *classes, int32_t *ranges,
+                   void *stream) {
+  if (key_mode != 0 && key_mode != 1) return SWA_ERR_INVALID_ARG;
+  if (B < 1 || n_q < 1 || W < 1) return SWA_ERR_INVALID_ARG;
+  if (key_mode == 0 && n_k < 1) return SWA_ERR_INVALID_ARG;
+  if (key_mode == 1 && (q_pos0 == nullptr || W >= (int64_t(1) << 40)))
+    return SWA_ERR_INVALID_ARG;
+  if (tile_q < 1 || tile_q > 1024 || tile_k < 1 || tile_k > 1024) return SWA_ERR_INVALID_ARG;
+  if (!classes && !ranges) return SWA_ERR_INVALID_ARG;
+  swa::MetaParams p;
+  p.key_mode = key_mode;
+  p.B = B;
+  p.n_q = n_q;
+  p.n_k = n_k;
+  p.W = W;
+  p.tile_q = tile_q;
+  p.tile_k = tile_k;
+  const int64_t nqt = (n_q + tile_q - 1) / tile_q;
+  const int64_t nkt = key_mode == 0 ? (n_k + tile_k - 1) / tile_k
+                                    : (W + tile_k - 1) / tile_k + (n_q + tile_k - 1) / tile_k;
+  if (nqt > 0x7FFFFFFF || nkt > 0x7FFFFFFF || B > 65535) return SWA_ERR_UNSUPPORTED;
+  p.nqt = static_cast<int>(nqt);
+  p.nkt = static_cast<int>(nkt);
+  p.q_pos0 = q_pos0;
+  p.classes = classes;
+  p.ranges = ranges;
+  dim3 grid(p.nqt, B);
+  swa::block_meta_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch();
+}
+
+int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                 int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream) {
+  int e = common_checks(B, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
+  if (N < 1 || N >= (int64_t(1) << 30)) return SWA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if ((e = make_map(&tq, q, d, N, static_cast<int64_t>(B) * H, kBQ))) return e;
+  if ((e = make_map(&tk, k, d, N, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  if ((e = make_map(&tv, v, d, N, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  swa::FwdParams p;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.q_start = nullptr;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.n_q = static_cast<int>(N);
+  p.n_k = static_cast<int>(N);
+  p.W = W < N + kBQ ? W : N + kBQ;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nqt = static_cast<int>((N + kBQ - 1) / kBQ);
+  p.n_ring_tiles = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_fwd<128, 0>(tq, tk, tv, tk, tv, p, st)
+                  : launch_fwd<64, 0>(tq, tk, tv, tk, tv, p, st);
+}
+
+int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_ring,
+                   const int64_t *q_start, int B, int Hkv, int64_t T, int d, int64_t W,
+                   void *stream) {
+  if (!k_new || !v_new || !k_ring || !v_ring || !q_start) return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hkv < 1 || T < 1 || W < 1 || (d != 64 && d != 128)) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) || !aligned16(v_ring))
+    return SWA_ERR_INVALID_ARG;
+  const int vec = d * 2 / 16;
+  const int64_t rows = T < W ? T : W;
+  const int64_t total = static_cast<int64_t>(B) * Hkv * rows * vec;
+  const int64_t blocks = (total + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  swa::ring_write_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
+      static_cast<uint4 *>(k_ring), static_cast<uint4 *>(v_ring), q_start, B, Hkv, T, vec, W);
+  return check_launch();
+}
+
+int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,
+                        void *v_ring, const int64_t *q_start, void *out, float *lse, int B,
+                        int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                        int update_ring, void *stream) {
+  int e = common_checks(B, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k_new || !v_new || !k_ring || !v_ring || !q_start || !out) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
+      !aligned16(v_ring) || !aligned16(out))
+    return SWA_ERR_INVALID_ARG;
+  if (Tq < 1 || Tq >= (int64_t(1) << 30) || W >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tkr, tvr;
+  if ((e = make_map(&tq, q, d, Tq, static_cast<int64_t>(B) * H, kBQ))) return e;
+  if ((e = make_map(&tk, k_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  if ((e = make_map(&tv, v_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  if ((e = make_map(&tkr, k_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  if ((e = make_map(&tvr, v_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  swa::FwdParams p;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.q_start = q_start;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.n_q = static_cast<int>(Tq);
+  p.n_k = static_cast<int>(Tq);
+  p.W = W;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nqt = static_cast<int>((Tq + kBQ - 1) / kBQ);
+  p.n_ring_tiles = static_cast<int>((W + kBK - 1) / kBK);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  e = d == 128 ? launch_fwd<128, 1>(tq, tk, tv, tkr, tvr, p, st)
+               : launch_fwd<64, 1>(tq, tk, tv, tkr, tvr, p, st);
+  if (e || !update_ring) return e;
+  return swa_ring_write(k_new, v_new, k_ring, v_ring, q_start, B, Hkv, Tq, d, W, stream);
+}
+
+size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int64_t W) {
+  if (B < 1 || H < 1 || Hkv < 1 || W < 1 || d < 1) return 0;
+  int chunk, splits;
+  decode_split(B, Hkv, W, &chunk, &splits);
+  const size_t rows = static_cast<size_t>(B) * H * splits;
+  return align256(rows * d * sizeof(float)) + align256(rows * 2 * sizeof(float));
+}
+
+int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
+                         const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
+                         int d, int64_t W, float scale, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+  int e = common_checks(B, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k_ring || !v_ring || !pos || !out) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out))
+    return SWA_ERR_INVALID_ARG;
+  if (W >= (int64_t(1) << 31) || B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+  const size_t need = swa_decode_workspace_bytes(B, H, Hkv, d, W);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SWA_ERR_WORKSPACE;
+  swa::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.k_ring = static_cast<const __nv_bfloat16 *>(k_ring);
+  p.v_ring = static_cast<const __nv_bfloat16 *>(v_ring);
+  p.pos = pos;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.W = W;
+  decode_split(B, Hkv, W, &p.chunk, &p.splits);
+  const size_t rows = static_cast<size_t>(B) * H * p.splits;
+  p.ws_o = static_cast<float *>(workspace);
+  p.ws_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                      align256(rows * d * sizeof(float)));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = H / Hkv;
+  return d == 128 ? dispatch_decode_g<128>(G, p, st) : dispatch_decode_g<64>(G, p, st);
+}
+
+int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,
+                            void *stream) {
+  if (B < 1 || W < 1 || !n_written || !slot_pos) return SWA_ERR_INVALID_ARG;
+  const int64_t total = static_cast<int64_t>(B) * W;
+  const int64_t blocks = (total + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  swa::ring_positions_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                               static_cast<cudaStream_t>(stream)>>>(B, n_written, W, slot_pos);
+  return check_launch();
+}
+
+int swa_get_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SWA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_swa_status, sizeof v) != cudaSuccess) return SWA_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_swa_status, &zero, sizeof zero) != cudaSuccess)
+    return SWA_ERR_CUDA;
+  if (v & SWA_DEV_TIMEOUT) return SWA_ERR_TIMEOUT;
+  if (v & SWA_DEV_BADARG) return SWA_ERR_DEVICE;
+  return SWA_OK;
+}
+
+}  // extern "C"

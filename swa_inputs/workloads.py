@@ -1,0 +1,78 @@
+"""The synthetic workloads: shapes, seeds and value recipes (no attention arithmetic).
+
+Every tensor is bf16 i.i.d. N(0, 1) from :func:`swa_inputs.normal_bf16` with the
+workload's seed and the tensor's own stream id.  Decode context lengths are
+uniform integers from the same generator.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import STREAM, normal_bf16, uniform_int
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str  # "prefill" | "chunk" | "decode"
+    B: int
+    H: int
+    Hkv: int
+    d: int
+    W: int
+    N: int = 0         # prefill sequence length
+    Tq: int = 0        # chunk length
+    q_start: int = 0   # chunk start (same for every sequence)
+    ctx_lo: int = 0    # decode context length range (inclusive)
+    ctx_hi: int = 0
+    seed: int = 0
+    note: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+# The five workloads (seed = index).
+WORKLOADS = {
+    "tiny": Workload("tiny", "prefill", B=1, H=4, Hkv=4, d=64, W=64, N=512, seed=0,
+                     note="tiny SWA forward, parity only"),
+    "mistral_prefill": Workload("mistral_prefill", "prefill", B=1, H=32, Hkv=8, d=128, W=4096,
+                                N=8192, seed=1, note="Mistral-7B-shaped prefill, GQA 4"),
+    "narrow_window": Workload("narrow_window", "prefill", B=2, H=32, Hkv=32, d=128, W=512,
+                              N=32768, seed=2, note="long prefill, narrow window"),
+    "chunk_ring": Workload("chunk_ring", "chunk", B=4, H=32, Hkv=8, d=128, W=4096, Tq=512,
+                           q_start=12288, seed=3, note="chunked prefill on a ring cache"),
+    "decode_ring": Workload("decode_ring", "decode", B=64, H=32, Hkv=8, d=128, W=4096,
+                            ctx_lo=4096, ctx_hi=131072, seed=4, note="batched decode"),
+}
+
+
+def prefill_inputs(w: Workload):
+    q = normal_bf16(w.seed, STREAM["q"], (w.B, w.H, w.N, w.d))
+    k = normal_bf16(w.seed, STREAM["k"], (w.B, w.Hkv, w.N, w.d))
+    v = normal_bf16(w.seed, STREAM["v"], (w.B, w.Hkv, w.N, w.d))
+    return q, k, v
+
+
+def chunk_inputs(w: Workload):
+    q = normal_bf16(w.seed, STREAM["q"], (w.B, w.H, w.Tq, w.d))
+    k_ring = normal_bf16(w.seed, STREAM["k_ring"], (w.B, w.Hkv, w.W, w.d))
+    v_ring = normal_bf16(w.seed, STREAM["v_ring"], (w.B, w.Hkv, w.W, w.d))
+    k_new = normal_bf16(w.seed, STREAM["k_new"], (w.B, w.Hkv, w.Tq, w.d))
+    v_new = normal_bf16(w.seed, STREAM["v_new"], (w.B, w.Hkv, w.Tq, w.d))
+    q_start = np.full(w.B, w.q_start, dtype=np.int64)
+    return q, k_new, v_new, k_ring, v_ring, q_start
+
+
+def decode_inputs(w: Workload):
+    q = normal_bf16(w.seed, STREAM["q"], (w.B, w.H, w.d))
+    k_ring = normal_bf16(w.seed, STREAM["k_ring"], (w.B, w.Hkv, w.W, w.d))
+    v_ring = normal_bf16(w.seed, STREAM["v_ring"], (w.B, w.Hkv, w.W, w.d))
+    ctx = uniform_int(w.seed, STREAM["ctx_len"], w.B, w.ctx_lo, w.ctx_hi)
+    pos = ctx - 1  # the query is the last token of its context
+    return q, k_ring, v_ring, pos

@@ -1,0 +1,130 @@
+"""swa_attn_chunk_ring (chunked prefill on a ring cache) and swa_ring_write vs the oracle."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import swa_inputs as si
+from swa_inputs.workloads import WORKLOADS, chunk_inputs
+from tests._util import assert_close, sample_rows, to_dev, to_f64, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def swa(cuda_ok):
+    import sliding_window_sparse_b200 as m
+
+    return m
+
+
+def _ring_from_history(seed, B, Hkv, W, d, q_starts):
+    """Ring contents after writing positions 0..q_start-1 (random rows per position)."""
+    rk = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rv = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    for b, qs in enumerate(q_starts):
+        if qs == 0:
+            continue
+        n = min(qs, W)
+        kk = si.normal_bf16(seed + b, si.STREAM["k_ring"], (1, Hkv, n, d))
+        vv = si.normal_bf16(seed + b, si.STREAM["v_ring"], (1, Hkv, n, d))
+        k1, v1 = oracle.ring_update(kk, vv, rk[b:b + 1], rv[b:b + 1], [qs - n], W)
+        rk[b:b + 1], rv[b:b + 1] = k1, v1
+    return rk, rv
+
+
+def _run(swa, q, kn, vn, rk, rv, qs, scale, update=False):
+    tq, tkn, tvn, trk, trv = (to_dev(x) for x in (q, kn, vn, rk, rv))
+    tqs = torch.tensor(qs, dtype=torch.int64, device="cuda")
+    out, lse = swa.swa_attn_chunk_ring(tq, tkn, tvn, trk, trv, tqs, scale, update_ring=update,
+                                       return_lse=True)
+    assert swa.swa_get_device_status() == 0
+    return out, lse, trk, trv
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,d,W,starts", [
+    (2, 4, 2, 64, 128, 256, [512, 600]),          # aligned and unaligned ring
+    (2, 4, 4, 200, 64, 128, [1000, 77]),          # chunk longer than the window
+    (3, 2, 1, 130, 128, 300, [0, 5, 301]),        # empty ring, partly filled, ragged tiles
+    (1, 8, 2, 1, 128, 64, [900]),                 # one-token chunk
+    (1, 4, 2, 384, 128, 512, [12288 + 37]),       # unaligned large start
+])
+def test_small_chunks_full_tensor(swa, B, H, Hkv, Tq, d, W, starts):
+    seed = 300 + Tq + W
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    scale = 1.0 / math.sqrt(d)
+    out, lse, trk, trv = _run(swa, q, kn, vn, rk, rv, starts, scale, update=True)
+    ref, ref_lse = oracle.swa_chunk(q, kn, vn, rk, rv, starts, W, scale, with_lse=True)
+    assert_close(to_f64(out), ref, what="chunk")
+    assert np.max(np.abs(to_f64(lse) - ref_lse)) < 1e-3
+    erk, erv = oracle.ring_update(kn, vn, rk, rv, starts, W)
+    assert np.array_equal(to_host_bits(trk), erk)
+    assert np.array_equal(to_host_bits(trv), erv)
+
+
+def test_chunk_workload_sampled_rows(swa):
+    w = WORKLOADS["chunk_ring"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    out, _, _, _ = _run(swa, q, kn, vn, rk, rv, list(qs), w.scale)
+    edges = [0, 1, 127, 128, 255, 256, 383, 384, 510, 511]
+    rows = sample_rows(w.B, w.H, w.Tq, 200, seed=11, extra=edges)
+    ref = oracle.swa_chunk(q, kn, vn, rk, rv, qs, w.W, w.scale, rows=rows)
+    got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert_close(got, ref, what="chunk_ring workload")
+
+
+def test_chunked_equals_full_prefill(swa):
+    """Chapter 10 section 10.5: full forward == chunks [0:2], [2:5], [5:7] through the ring
+    (7 tokens, W = 3), and the same on a larger case with ragged chunks."""
+    for N, W, chunks in [(7, 3, [(0, 2), (2, 5), (5, 7)]),
+                         (700, 200, [(0, 100), (100, 101), (101, 450), (450, 700)])]:
+        B, H, Hkv, d = 1, 4, 2, 128
+        q = si.normal_bf16(9, si.STREAM["q"], (B, H, N, d))
+        k = si.normal_bf16(9, si.STREAM["k"], (B, Hkv, N, d))
+        v = si.normal_bf16(9, si.STREAM["v"], (B, Hkv, N, d))
+        full = to_f64(swa.swa_attn_fwd(to_dev(q), to_dev(k), to_dev(v), W, 0.1))
+        rk = torch.zeros((B, Hkv, W, d), dtype=torch.bfloat16, device="cuda")
+        rv = torch.zeros_like(rk)
+        parts = []
+        for c0, c1 in chunks:
+            qs = torch.tensor([c0], dtype=torch.int64, device="cuda")
+            o = swa.swa_attn_chunk_ring(to_dev(np.ascontiguousarray(q[:, :, c0:c1])),
+                                        to_dev(np.ascontiguousarray(k[:, :, c0:c1])),
+                                        to_dev(np.ascontiguousarray(v[:, :, c0:c1])),
+                                        rk, rv, qs, 0.1, update_ring=True)
+            parts.append(to_f64(o))
+        chunked = np.concatenate(parts, axis=2)
+        assert_close(chunked, full, what=f"chunked N{N}")
+        ref = oracle.swa_forward(q, k, v, W, 0.1)
+        assert_close(chunked, ref, what="chunked vs oracle")
+
+
+def test_ring_write_bit_exact(swa):
+    B, Hkv, T, d, W = 3, 2, 70, 64, 32
+    kn = si.normal_bf16(1, 6, (B, Hkv, T, d))
+    vn = si.normal_bf16(1, 7, (B, Hkv, T, d))
+    rk = si.normal_bf16(1, 4, (B, Hkv, W, d))
+    rv = si.normal_bf16(1, 5, (B, Hkv, W, d))
+    starts = [0, 31, 1000]
+    trk, trv = to_dev(rk), to_dev(rv)
+    swa.swa_ring_write(to_dev(kn), to_dev(vn), trk, trv,
+                       torch.tensor(starts, dtype=torch.int64, device="cuda"))
+    erk, erv = oracle.ring_update(kn, vn, rk, rv, starts, W)
+    assert np.array_equal(to_host_bits(trk), erk)
+    assert np.array_equal(to_host_bits(trv), erv)
+
+
+def test_negative_start_reports_device_error(swa):
+    B, H, Hkv, Tq, d, W = 1, 2, 2, 16, 64, 32
+    z = torch.zeros((B, H, Tq, d), dtype=torch.bfloat16, device="cuda")
+    zk = torch.zeros((B, Hkv, Tq, d), dtype=torch.bfloat16, device="cuda")
+    rk = torch.zeros((B, Hkv, W, d), dtype=torch.bfloat16, device="cuda")
+    qs = torch.tensor([-1], dtype=torch.int64, device="cuda")
+    swa.swa_attn_chunk_ring(z, zk, zk, rk, rk.clone(), qs, 0.1)
+    assert swa.swa_get_device_status() == 6
