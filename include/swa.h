@@ -100,7 +100,7 @@ SWA_API int swa_block_meta(int key_mode, int B, int64_t n_q, int64_t n_k, const 
  *        scaled scores of each row over its allowed keys.
  * Query and key row i both sit at logical position i.  Only key tiles that
  * hold an allowed pair are loaded; only partially visible tiles are masked.
- * Limits: 1 <= N < 2^30, H % Hkv == 0.
+ * Limits: 1 <= N < 2^29, H % Hkv == 0.
  */
 SWA_API int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
                  int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream);
@@ -123,7 +123,7 @@ SWA_API int swa_attn_fwd(const void *q, const void *k, const void *v, void *out,
  * logical position.  If update_ring != 0, after the attention (same stream)
  * the chunk rows whose positions are among the last W are written into slots
  * position mod W, so the ring then serves the next chunk or decode step.
- * The ring is only written when update_ring != 0.  Limits: 1 <= Tq < 2^30,
+ * The ring is only written when update_ring != 0.  Limits: 1 <= Tq < 2^29,
  * W < 2^29.
  */
 SWA_API int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,

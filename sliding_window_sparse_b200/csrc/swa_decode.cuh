@@ -2,19 +2,22 @@
 //
 // The cost of a decode step is reading the KV cache from HBM (sparse-attention
 // taxonomy page, section 1), so the split kernel streams every key/value slot
-// of a (sequence, kv head) exactly once, with coalesced 8-byte (d = 128) or
-// 4-byte (d = 64) loads per lane, and serves all G query heads of the group
-// from the same registers.  The slot range of one (b, kv head) is cut into
-// `splits` CTAs; each writes an unnormalised partial (o, running max m,
-// running sum l) to the workspace, and decode_combine_kernel merges them.
+// of a (sequence, kv head) exactly once with 16-byte coalesced loads and serves
+// all G query heads of the group from the same registers.  The slot range of
+// one (b, kv head) is cut into `splits` CTAs; each writes an unnormalised
+// partial (o, running max m, running sum l, base 2) to the workspace, and
+// decode_combine_kernel merges them.
 //
-// Warp layout: lane owns DPL = d / 32 consecutive dims of q, k, v and o.
-// A warp takes KEYS = 32 / G keys at a time: it forms the 32 partial dot
-// products (key, head) of its lane slice, then a butterfly reduce-scatter
-// over the 32 lanes leaves lane l with the full score of key l / G for head
-// l % G.  Online softmax (base 2, scale * log2(e) folded into q) runs per
-// head across the lanes that hold that head; the probabilities are staged in
-// shared memory and every lane accumulates its o slice.
+// Warp layout: a key row of D bf16 is read by LPK = D / 8 lanes (16 bytes
+// each), so one warp-wide load covers KPW = 32 / LPK consecutive slots.  Lane
+// (kg, sub) owns head dims [8 sub, 8 sub + 8) of the keys kg, kg + KPW, ...
+// A step takes R loads per lane (KPS = R * KPW slots).  The lane forms
+// NV = R * G partial dot products (its 8 dims, packed f32x2 FMAs); a butterfly
+// over the LPK lanes of its key group scatters them so that lane sub ends with
+// the full score of value index sub / DUP (DUP = LPK / NV lanes hold each
+// value).  Online softmax per head runs across the lanes holding that head;
+// probabilities go through shared memory and every lane accumulates the
+// partial o of its keys and dims; the KPW key groups are summed at the end.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -41,59 +44,54 @@ struct DecodeParams {
   float scale_log2;
 };
 
-template <int DPL>
-struct RowVec;
-template <>
-struct RowVec<4> {
-  using T = uint2;
-};
-template <>
-struct RowVec<2> {
-  using T = uint32_t;
-};
-
-template <int DPL>
-__device__ __forceinline__ void unpack_row(const typename RowVec<DPL>::T &raw, float (&f)[DPL]);
-template <>
-__device__ __forceinline__ void unpack_row<4>(const uint2 &raw, float (&f)[4]) {
-  f[0] = __uint_as_float(raw.x << 16);
-  f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-  f[2] = __uint_as_float(raw.y << 16);
-  f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ void unpack_row<2>(const uint32_t &raw, float (&f)[2]) {
-  f[0] = __uint_as_float(raw << 16);
-  f[1] = __uint_as_float(raw & 0xFFFF0000u);
+__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 &raw, float2 (&f)[4]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
-template <int DPL>
-__device__ __forceinline__ typename RowVec<DPL>::T load_row_nc(const __nv_bfloat16 *p) {
-  using T = typename RowVec<DPL>::T;
-  return __ldg(reinterpret_cast<const T *>(p));
+__device__ __forceinline__ uint4 ldg_stream(const __nv_bfloat16 *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecWarps * 32)
-    decode_split_kernel(const DecodeParams p) {
-  constexpr int DPL = D / 32;
-  constexpr int KEYS = 32 / G;  // keys per warp step: KEYS * G == 32 (key, head) scores
-  using Raw = typename RowVec<DPL>::T;
+struct DecodeShape {
+  static constexpr int LPK = D / 8;                       // lanes per key row
+  static constexpr int KPW = 32 / LPK;                    // slots per warp-wide load
+  static constexpr int MAXR = D == 128 ? 4 : 2;
+  static constexpr int R = (LPK / G) < MAXR ? (LPK / G) : MAXR;  // loads per lane per step
+  static constexpr int NV = R * G;                        // partial dots per lane
+  static constexpr int DUP = LPK / NV;                    // lanes holding each full value
+  static constexpr int KPS = R * KPW;                     // slots per step
+  static_assert(R >= 1 && NV <= LPK && (LPK % NV) == 0, "unsupported group size");
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const DecodeParams p) {
+  using S = DecodeShape<D, G>;
+  constexpr int LPK = S::LPK, KPW = S::KPW, R = S::R, NV = S::NV, DUP = S::DUP, KPS = S::KPS;
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int sub = lane % LPK;  // dims [8 sub, 8 sub + 8)
+  const int kg = lane / LPK;   // key group within a warp-wide load
 
-  __shared__ float s_p[kDecWarps][32];
+  __shared__ float s_p[kDecWarps][KPS * G];
   __shared__ float s_alpha[kDecWarps][G];
   __shared__ float s_m[kDecWarps][G];
   __shared__ float s_l[kDecWarps][G];
   __shared__ float s_o[kDecWarps][G][D];
 
   const int64_t pos = p.pos[b];
-  int64_t nvalid = pos + 1 < p.W ? pos + 1 : p.W;  // slots 0..pos are filled before wrap
+  int64_t nvalid = pos + 1 < p.W ? pos + 1 : p.W;  // slots 0..pos are filled before the wrap
   if (pos < 0) {
     nvalid = 0;
     if (threadIdx.x == 0 && split == 0 && kvh == 0) atomicOr(&g_swa_status, SWA_DEV_BADARG);
@@ -102,126 +100,157 @@ __global__ void __launch_bounds__(kDecWarps * 32)
   int64_t s_end = s_begin + p.chunk;
   if (s_end > nvalid) s_end = nvalid;
 
-  // q slices of the G heads of this group, pre-scaled into the base-2 domain
-  float qv[G][DPL];
+  // q slices of the G heads (8 dims each), pre-scaled into the base-2 domain
+  float2 qv[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16 *qp = p.q + (static_cast<int64_t>(b) * p.H + kvh * G + g) * D + lane * DPL;
-    float f[DPL];
-    unpack_row<DPL>(load_row_nc<DPL>(qp), f);
+    const __nv_bfloat16 *qp = p.q + (static_cast<int64_t>(b) * p.H + kvh * G + g) * D + sub * 8;
+    float2 f[4];
+    bf16x8_to_f32x2(*reinterpret_cast<const uint4 *>(qp), f);
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) qv[g][i] = f[i] * p.scale_log2;
+    for (int i = 0; i < 4; ++i) qv[g][i] = make_float2(f[i].x * p.scale_log2, f[i].y * p.scale_log2);
   }
 
   const int64_t kv_base = (static_cast<int64_t>(b) * p.Hkv + kvh) * p.W;
-  const __nv_bfloat16 *kbase = p.k_ring + kv_base * D + lane * DPL;
-  const __nv_bfloat16 *vbase = p.v_ring + kv_base * D + lane * DPL;
+  const __nv_bfloat16 *kbase = p.k_ring + kv_base * D + sub * 8;
+  const __nv_bfloat16 *vbase = p.v_ring + kv_base * D + sub * 8;
 
-  float o[G][DPL];
+  float2 o[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) o[g][i] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;  // for head (lane % G)
+    for (int i = 0; i < 4; ++i) o[g][i] = make_float2(0.f, 0.f);
+  float m_run = -INFINITY, l_run = 0.f;  // head of this lane's value index
 
-  // warp w takes steps w, w + 4, ...; a step covers KEYS consecutive slots
-  const int64_t n_steps = s_end > s_begin ? (s_end - s_begin + KEYS - 1) / KEYS : 0;
-  Raw kr[KEYS], vr[KEYS];
-  auto load_step = [&](int64_t step, Raw (&kk)[KEYS], Raw (&vv)[KEYS]) {
-    const int64_t s0 = s_begin + step * KEYS;
+  const int64_t n_steps = s_end > s_begin ? (s_end - s_begin + KPS - 1) / KPS : 0;
+  uint4 kr[R], vr[R];
+  auto load_step = [&](int64_t step, uint4 (&kk)[R], uint4 (&vv)[R]) {
+    const int64_t s0 = s_begin + step * KPS + kg;
 #pragma unroll
-    for (int k = 0; k < KEYS; ++k) {
-      int64_t s = s0 + k;
+    for (int r = 0; r < R; ++r) {
+      int64_t s = s0 + r * KPW;
       if (s >= s_end) s = s_begin;  // in-bounds dummy, masked below
-      kk[k] = load_row_nc<DPL>(kbase + s * D);
-      vv[k] = load_row_nc<DPL>(vbase + s * D);
+      kk[r] = ldg_stream(kbase + s * D);
+      vv[r] = ldg_stream(vbase + s * D);
     }
   };
   int64_t step = warp;
   if (step < n_steps) load_step(step, kr, vr);
   for (; step < n_steps; step += kDecWarps) {
-    Raw kc[KEYS], vc[KEYS];
+    uint4 kc[R], vc[R];
 #pragma unroll
-    for (int k = 0; k < KEYS; ++k) {
-      kc[k] = kr[k];
-      vc[k] = vr[k];
+    for (int r = 0; r < R; ++r) {
+      kc[r] = kr[r];
+      vc[r] = vr[r];
     }
     if (step + kDecWarps < n_steps) load_step(step + kDecWarps, kr, vr);
 
-    // partial dots of this lane's slice: part[k * G + g]
-    float part[32];
+    // partial dot products part[r * G + g] over this lane's 8 dims
+    float part[NV];
 #pragma unroll
-    for (int k = 0; k < KEYS; ++k) {
-      float kf[DPL];
-      unpack_row<DPL>(kc[k], kf);
+    for (int r = 0; r < R; ++r) {
+      float2 kf[4];
+      bf16x8_to_f32x2(kc[r], kf);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float acc = 0.f;
+        float2 acc = __fmul2_rn(qv[g][0], kf[0]);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) acc = fmaf(qv[g][i], kf[i], acc);
-        part[k * G + g] = acc;
+        for (int i = 1; i < 4; ++i) acc = __ffma2_rn(qv[g][i], kf[i], acc);
+        part[r * G + g] = acc.x + acc.y;
       }
     }
-    // butterfly reduce-scatter: lane l ends with the full value of index l
+    // butterfly over the LPK lanes of the key group: scatter NV values, then sum duplicates
+    {
+      int cnt = NV;
 #pragma unroll
-    for (int half = 16; half >= 1; half >>= 1) {
-      const bool upper = (lane & half) != 0;
+      for (int half = LPK / 2; half >= 1; half >>= 1) {
+        if (cnt > 1) {
+          const int h2 = cnt / 2;
+          const bool upper = (sub & half) != 0;
 #pragma unroll
-      for (int i = 0; i < half; ++i) {
-        const float keep = upper ? part[i + half] : part[i];
-        const float send = upper ? part[i] : part[i + half];
-        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+          for (int i = 0; i < NV / 2; ++i) {
+            if (i < h2) {
+              const float keep = upper ? part[i + h2] : part[i];
+              const float send = upper ? part[i] : part[i + h2];
+              part[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+            }
+          }
+          cnt = h2;
+        } else {
+          part[0] += __shfl_xor_sync(0xffffffffu, part[0], half);
+        }
       }
     }
-    const int my_key = lane / G;
-    const int64_t my_slot = s_begin + step * KEYS + my_key;
-    float sc = my_slot < s_end ? part[0] : -INFINITY;
-    // max and sum per head over the lanes holding that head (xor masks >= G)
+    const int v_idx = sub / DUP;  // value index held by this lane
+    const int my_r = v_idx / G, my_g = v_idx % G;
+    const int key_in_step = my_r * KPW + kg;
+    const int64_t my_slot = s_begin + step * KPS + key_in_step;
+    const float sc = my_slot < s_end ? part[0] : -INFINITY;
+    // max and sum per head over the lanes holding that head (one copy per value)
     float mx = sc;
 #pragma unroll
-    for (int m = G; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    for (int m = DUP * G; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
     const float m_new = fmaxf(m_run, mx);
     const float m_use = m_new == -INFINITY ? 0.f : m_new;
     const float alpha = ex2(m_run - m_use);  // m_run = -inf gives 0
     const float pr = ex2(sc - m_use);        // masked score gives 0
     float ps = pr;
 #pragma unroll
-    for (int m = G; m < 32; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
+    for (int m = DUP * G; m < 32; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
     l_run = l_run * alpha + ps;
     m_run = m_new;
 
-    s_p[warp][lane] = pr;
-    if (lane < G) s_alpha[warp][lane] = alpha;
+    s_p[warp][key_in_step * G + my_g] = pr;
+    if (kg == 0 && v_idx < G) s_alpha[warp][v_idx] = alpha;
     __syncwarp();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float a = s_alpha[warp][g];
+      const float2 a2 = make_float2(a, a);
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) o[g][i] *= a;
+      for (int i = 0; i < 4; ++i) o[g][i] = __fmul2_rn(o[g][i], a2);
     }
 #pragma unroll
-    for (int k = 0; k < KEYS; ++k) {
-      float vf[DPL];
-      unpack_row<DPL>(vc[k], vf);
+    for (int r = 0; r < R; ++r) {
+      float2 vf[4];
+      bf16x8_to_f32x2(vc[r], vf);
+      const int key = r * KPW + kg;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float pk = s_p[warp][k * G + g];
+        const float pk = s_p[warp][key * G + g];
+        const float2 p2 = make_float2(pk, pk);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(pk, vf[i], o[g][i]);
+        for (int i = 0; i < 4; ++i) o[g][i] = __ffma2_rn(p2, vf[i], o[g][i]);
       }
     }
     __syncwarp();
   }
 
-  // merge the four warps of this CTA
-  if (lane < G) {
-    s_m[warp][lane] = m_run;
-    s_l[warp][lane] = l_run;
+  // sum the partial o of the KPW key groups (same dims, different slots)
+#pragma unroll
+  for (int m = LPK; m < 32; m <<= 1)
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[g][i].x += __shfl_xor_sync(0xffffffffu, o[g][i].x, m);
+        o[g][i].y += __shfl_xor_sync(0xffffffffu, o[g][i].y, m);
+      }
+  // merge the warps of this CTA (a lane of key group 0 whose value index g < G holds head g's m, l)
+  if (kg == 0 && sub / DUP < G) {
+    const int g = sub / DUP;
+    s_m[warp][g] = m_run;
+    s_l[warp][g] = l_run;
   }
+  if (kg == 0) {
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) s_o[warp][g][lane * DPL + i] = o[g][i];
+      for (int i = 0; i < 4; ++i) {
+        s_o[warp][g][sub * 8 + 2 * i] = o[g][i].x;
+        s_o[warp][g][sub * 8 + 2 * i + 1] = o[g][i].y;
+      }
+  }
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, c = idx % D;

@@ -1,0 +1,551 @@
+// swa_fwd2.cuh -- persistent, two-query-tile sliding-window attention forward
+// for sm_100a (tcgen05 MMAs, tensor-memory accumulators, TMA staging).
+//
+// Work unit: two 128-row query tiles A and B that read the same key/value
+// tiles.  With G = H / Hkv even they are two query heads of one key/value
+// group at the same query rows (identical tile lists); otherwise they are
+// query tiles 2p and 2p+1 of one head (the key stream is the union of both
+// windows and each tile uses its own part).  CTAs are persistent: CTA c takes
+// units c, c + gridDim.x, ... (heavy query tiles first).
+//
+// Roles (320 threads):
+//   warp 0      TMA producer: Q_A, Q_B once per unit, then K/V tiles into a
+//               2-stage shared-memory ring (128-byte swizzle, one box per 64
+//               head-dim columns).  Only live key tiles are loaded (M003 note
+//               section 04).
+//   warp 1      one thread issues every tcgen05.mma:
+//                 S_X = Q_X K^T        (A, B from shared memory)
+//                 O_X += P_X V         (P from tensor memory, V from shared memory)
+//               in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
+//               softmax of one tile overlaps the MMAs of the other.
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one row per
+//               thread, one tensor-memory lane quadrant per warp.  Mask only
+//               partial or ragged tiles, base-2 exponentials with
+//               scale * log2(e) folded in, running max and sum in fp32, P
+//               packed to bf16 into the tile's S columns, O rescaled in tensor
+//               memory only when the running max grows by more than 2^8.
+//               After the unit's last tile: O / l to bf16 rows, and the
+//               log-sum-exp.
+//
+// Tensor memory (512 columns): S_A/P_A [0,128), S_B/P_B [128,256),
+// O_A [256, 256+D), O_B [256+D, 256+2D).  P_X overwrites the first 64 columns
+// of S_X; the next S_X is issued after PV_X, and tcgen05 MMAs issued by one
+// thread execute in order.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+#include "swa_tile.cuh"
+
+namespace swa {
+
+constexpr int kQT = 128;  // query rows per tile (MMA M, tensor-memory lanes)
+constexpr int kKT = 128;  // keys per tile
+constexpr int kFwd2Threads = 320;
+constexpr float kLazyRescaleLog2 = 8.0f;
+
+struct Fwd2Params {
+  __nv_bfloat16 *out;      // [B, H, n_q, D]
+  float *lse;              // [B, H, n_q] or nullptr
+  const int64_t *q_start;  // MODE 1: [B]
+  int B, H, Hkv, G;
+  int n_q;                 // query rows per (b, h)
+  int n_k;                 // rows of the main key source (N, or Tq for a chunk)
+  int64_t W;               // window (MODE 0: clamped to n_k + kQT)
+  float scale_log2;        // scale * log2(e)
+  int nqt;                 // query tiles per (b, h)
+  int n_ring_tiles;        // MODE 1: ceil(W / kKT)
+  int pair_heads;          // 1: A/B are heads 2p, 2p+1 of a group; 0: q tiles 2p, 2p+1
+  int n_units;
+};
+
+template <int D>
+struct Fwd2Layout {
+  static constexpr int PANELS = D / 64;
+  static constexpr int NST = D == 64 ? 4 : 2;
+  static constexpr uint32_t Q_BYTES = kQT * D * 2;
+  static constexpr uint32_t KV_BYTES = kKT * D * 2;
+  static constexpr uint32_t OFF_QA = 0;
+  static constexpr uint32_t OFF_QB = Q_BYTES;
+  static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + NST * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NST * KV_BYTES;
+  // q_full, q_empty, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2], o_full[2]
+  static constexpr int NBAR = 2 + 3 * NST + 6;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t BYTES = OFF_MISC + 16;
+  static constexpr uint32_t ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+struct Unit {
+  int b, kvh, h[2], t[2];
+  bool has_b;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const Fwd2Params &p) {
+  Unit U;
+  if (p.pair_heads) {
+    const int half = p.G >> 1;
+    const int per_t = p.B * p.Hkv * half;
+    const int t = p.nqt - 1 - u / per_t;
+    const int r = u % per_t;
+    const int pair = r % half, bk = r / half;
+    U.b = bk / p.Hkv;
+    U.kvh = bk % p.Hkv;
+    U.h[0] = U.kvh * p.G + 2 * pair;
+    U.h[1] = U.h[0] + 1;
+    U.t[0] = U.t[1] = t;
+    U.has_b = true;
+  } else {
+    const int npairs = (p.nqt + 1) >> 1;
+    const int pr = npairs - 1 - u % npairs;
+    const int bh = u / npairs;
+    U.b = bh / p.H;
+    U.h[0] = U.h[1] = bh % p.H;
+    U.kvh = U.h[0] / p.G;
+    U.t[0] = 2 * pr;
+    U.t[1] = 2 * pr + 1;
+    U.has_b = U.t[1] < p.nqt;
+  }
+  return U;
+}
+
+// Live key tiles of a unit in stream order, with the class for each query
+// tile.  Positions are int32: MODE 0 uses absolute positions (< 2^30),
+// MODE 1 positions relative to the chunk start (ring slots hold -W .. -1).
+// The segment bases follow the ring layout of swa_tile.cuh.
+template <int MODE>
+struct Walker2 {
+  int kt, kt_end;
+  int qlo[2], qhi[2];
+  int W;         // MODE 0: clamped window; MODE 1: ring slots
+  int n_k;       // MODE 0 key rows; MODE 1 chunk rows
+  int nrt;       // MODE 1 ring tiles
+  int wrap;      // MODE 1: ring full ? L mod W : number of filled slots
+  bool full_ring;
+  bool has_b;
+
+  __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs) {
+    has_b = U.has_b;
+    n_k = p.n_k;
+    W = static_cast<int>(p.W);
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      qlo[x] = U.t[x] * kQT;
+      qhi[x] = min(qlo[x] + kQT, p.n_q) - 1;
+    }
+    if (MODE == 0) {
+      kt = max(qlo[0] - (W - 1), 0) / kKT;
+      kt_end = (has_b ? qhi[1] : qhi[0]) / kKT + 1;
+      nrt = 0;
+      wrap = 0;
+      full_ring = false;
+    } else {
+      nrt = p.n_ring_tiles;
+      kt = 0;
+      kt_end = nrt + (p.n_q + kKT - 1) / kKT;
+      full_ring = qs >= p.W;
+      wrap = static_cast<int>(full_ring ? qs % p.W : qs);
+    }
+  }
+
+  // Segments of tile kt: columns [lo_g, hi_g] hold positions base_g + c.
+  __device__ __forceinline__ int segments(int k, int (&lo)[2], int (&hi)[2], int (&base)[2],
+                                          int &src, int &y0) const {
+    lo[1] = 1;
+    hi[1] = 0;
+    base[1] = 0;
+    if (MODE == 0 || k >= nrt) {
+      const int c0 = (k - nrt) * kKT;
+      const int nc = min(kKT, n_k - c0);
+      src = 0;
+      y0 = c0;
+      lo[0] = 0;
+      hi[0] = nc - 1;
+      base[0] = c0;
+      return nc;
+    }
+    const int s0 = k * kKT;
+    const int nc = min(kKT, W - s0);
+    src = 1;
+    y0 = s0;
+    if (!full_ring) {  // slots 0 .. wrap-1 hold positions 0 .. wrap-1 (relative: s - wrap)
+      lo[0] = 0;
+      hi[0] = min(nc - 1, wrap - 1 - s0);
+      base[0] = s0 - wrap;
+    } else {  // slots < wrap: position s - wrap; slots >= wrap: s - wrap - W
+      lo[0] = 0;
+      hi[0] = min(nc - 1, wrap - 1 - s0);
+      base[0] = s0 - wrap;
+      lo[1] = max(0, wrap - s0);
+      hi[1] = nc - 1;
+      base[1] = s0 - wrap - W;
+    }
+    return nc;
+  }
+
+  __device__ __forceinline__ int klass(int x, int nc, const int (&lo)[2], const int (&hi)[2],
+                                       const int (&base)[2]) const {
+    bool any = false;
+    int all_cols = 0;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      if (lo[g] > hi[g]) continue;
+      const int p_lo = base[g] + lo[g], p_hi = base[g] + hi[g];
+      if (p_lo <= qhi[x] && p_hi + W - 1 >= qlo[x]) any = true;
+      if (p_hi <= qlo[x] && p_lo >= qhi[x] - W + 1) all_cols += hi[g] - lo[g] + 1;
+    }
+    // A ragged tile (nc < kKT) is masked even when every in-range pair is allowed:
+    // its out-of-range columns read as zero and must not enter the softmax.
+    return !any ? 0 : (all_cols == nc && nc == kKT ? 1 : 2);
+  }
+
+  // Advance to the next live tile: its index, source, first row and classes.
+  __device__ __forceinline__ bool next(int &k, int &src, int &y0, int &ca, int &cb) {
+    while (kt < kt_end) {
+      k = kt++;
+      int lo[2], hi[2], base[2];
+      const int nc = segments(k, lo, hi, base, src, y0);
+      ca = klass(0, nc, lo, hi, base);
+      cb = has_b ? klass(1, nc, lo, hi, base) : 0;
+      if (ca | cb) return true;
+    }
+    return false;
+  }
+};
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kFwd2Threads, 1)
+    fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_vr, const Fwd2Params p) {
+  using L = Fwd2Layout<D>;
+  constexpr int NST = L::NST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (base - raw);
+  const uint32_t sQ[2] = {base + L::OFF_QA, base + L::OFF_QB};
+  const uint32_t sK = base + L::OFF_K, sV = base + L::OFF_V, bar = base + L::OFF_BAR;
+  const uint32_t BAR_QF = bar, BAR_QE = bar + 8;
+  const uint32_t BAR_KF = bar + 16;                 // + 8 * stage
+  const uint32_t BAR_VF = bar + 16 + 8 * NST;       // + 8 * stage
+  const uint32_t BAR_KVE = bar + 16 + 16 * NST;     // + 8 * stage
+  const uint32_t BAR_S = bar + 16 + 24 * NST;       // + 8 * tile
+  const uint32_t BAR_P = BAR_S + 16;                // + 8 * tile
+  const uint32_t BAR_O = BAR_P + 16;                // + 8 * tile
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_QF, 1);
+    mbar_init(BAR_QE, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(BAR_KF + 8 * s, 1);
+      mbar_init(BAR_VF + 8 * s, 1);
+      mbar_init(BAR_KVE + 8 * s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(BAR_S + 8 * x, 1);
+      mbar_init(BAR_P + 8 * x, 4 * 32);
+      mbar_init(BAR_O + 8 * x, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    if (MODE == 1) {
+      tma_prefetch_desc(&tm_kr);
+      tma_prefetch_desc(&tm_vr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto unit_start = [&](const Unit &U, int64_t &qs) -> bool {
+    qs = 0;
+    if (MODE == 1) {
+      qs = p.q_start[U.b];
+      if (qs < 0) return false;
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kv_iter = 0, q_iter = 0;
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const Unit U = decode_unit(u, p);
+        int64_t qs;
+        if (!unit_start(U, qs)) {
+          atomicOr(&g_swa_status, SWA_DEV_BADARG);
+          continue;
+        }
+        if (q_iter > 0 && !mbar_wait(BAR_QE, (q_iter - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(BAR_QF, (U.has_b ? 2u : 1u) * L::Q_BYTES);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x == 1 && !U.has_b) break;
+#pragma unroll
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_3d(sQ[x] + pn * (kQT * 128), &tm_q, BAR_QF, pn * 64, U.t[x] * kQT,
+                        U.b * p.H + U.h[x]);
+        }
+        ++q_iter;
+        Walker2<MODE> wk;
+        wk.init(U, p, qs);
+        int k, src, y0, ca, cb;
+        const int z = U.b * p.Hkv + U.kvh;
+        while (wk.next(k, src, y0, ca, cb)) {
+          const int st = kv_iter % NST;
+          if (kv_iter >= NST && !mbar_wait(BAR_KVE + 8 * st, ((kv_iter / NST) - 1) & 1, abort_flag))
+            break;
+          const CUtensorMap *mk = src == 1 ? &tm_kr : &tm_k;
+          const CUtensorMap *mv = src == 1 ? &tm_vr : &tm_v;
+          mbar_expect_tx(BAR_KF + 8 * st, L::KV_BYTES);
+#pragma unroll
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_3d(sK + st * L::KV_BYTES + pn * (kKT * 128), mk, BAR_KF + 8 * st, pn * 64,
+                        y0, z);
+          mbar_expect_tx(BAR_VF + 8 * st, L::KV_BYTES);
+#pragma unroll
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_3d(sV + st * L::KV_BYTES + pn * (kKT * 128), mv, BAR_VF + 8 * st, pn * 64,
+                        y0, z);
+          ++kv_iter;
+        }
+        if (*abort_flag) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kQT, kKT, false);
+      constexpr uint32_t idO = idesc_bf16_f32(kQT, D, true);
+      int kv_iter = 0, q_iter = 0;
+      uint32_t p_cnt[2] = {0u, 0u};
+      auto issue_s = [&](int x, int st) {
+        const uint32_t dS = tmem + x * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offq = (kk >> 2) * (kQT * 128) + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * (kKT * 128) + (kk & 3) * 32;
+          mma_ss(dS, sdesc_sw128(sQ[x] + offq, 16, 1024),
+                 sdesc_sw128(sK + st * L::KV_BYTES + offk, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR_S + 8 * x);
+      };
+      auto issue_pv = [&](int x, int st, bool acc) {
+        const uint32_t dO = tmem + 256 + x * D;
+        const uint32_t aP = tmem + x * 128;
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk)
+          mma_ts(dO, aP + kk * 8, sdesc_sw128(sV + st * L::KV_BYTES + kk * 16 * 128, kKT * 128, 1024),
+                 idO, (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const Unit U = decode_unit(u, p);
+        int64_t qs;
+        if (!unit_start(U, qs)) continue;
+        mbar_wait(BAR_QF, q_iter & 1, abort_flag);
+        tc_fence_after();
+        Walker2<MODE> wk;
+        wk.init(U, p, qs);
+        int k, src, y0, ca, cb;
+        bool have = wk.next(k, src, y0, ca, cb);
+        bool first[2] = {true, true};
+        if (have) {
+          const int st = kv_iter % NST;
+          mbar_wait(BAR_KF + 8 * st, (kv_iter / NST) & 1, abort_flag);
+          tc_fence_after();
+          if (ca) issue_s(0, st);
+          if (cb) issue_s(1, st);
+        } else {
+          tc_commit(BAR_QE);
+        }
+        while (have) {
+          int na = 0, nb = 0;
+          const bool has_next = wk.next(k, src, y0, na, nb);
+          if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
+          const int st = kv_iter % NST;
+          const int stn = (kv_iter + 1) % NST;
+          mbar_wait(BAR_VF + 8 * st, (kv_iter / NST) & 1, abort_flag);
+          if (has_next) mbar_wait(BAR_KF + 8 * stn, ((kv_iter + 1) / NST) & 1, abort_flag);
+          if (ca) {
+            mbar_wait(BAR_P, p_cnt[0] & 1, abort_flag);
+            ++p_cnt[0];
+            tc_fence_after();
+            issue_pv(0, st, !first[0]);
+            first[0] = false;
+          }
+          if (has_next && na) issue_s(0, stn);
+          if (cb) {
+            mbar_wait(BAR_P + 8, p_cnt[1] & 1, abort_flag);
+            ++p_cnt[1];
+            tc_fence_after();
+            issue_pv(1, st, !first[1]);
+            first[1] = false;
+          }
+          if (has_next && nb) issue_s(1, stn);
+          tc_commit(BAR_KVE + 8 * st);
+          ++kv_iter;
+          ca = na;
+          cb = nb;
+          have = has_next;
+        }
+        tc_commit(BAR_O);
+        tc_commit(BAR_O + 8);
+        ++q_iter;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int x = warp < 6 ? 0 : 1;  // query tile of this warp group
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + x * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + x * D + lane_off;
+    uint32_t s_cnt = 0, u_iter = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      const Unit U = decode_unit(u, p);
+      int64_t qs;
+      if (!unit_start(U, qs)) continue;
+      Walker2<MODE> wk;
+      wk.init(U, p, qs);
+      const int qrow = U.t[x] * kQT + row;  // MODE 0 absolute, MODE 1 relative to q_start
+      float m_run = -INFINITY, l_run = 0.f;
+      int nt = 0;
+      int k, src, y0, ca, cb;
+      while (wk.next(k, src, y0, ca, cb)) {
+        const int cls = x == 0 ? ca : cb;
+        if (!cls) continue;
+        mbar_wait(BAR_S + 8 * x, s_cnt & 1, abort_flag);
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld128(tS, sr);
+        float *s = reinterpret_cast<float *>(sr);
+        if (cls == 2) {
+          // allowed columns of this row: c in a segment with base + c in [q - W + 1, q]
+          int lo[2], hi[2], base[2], s_, y_;
+          wk.segments(k, lo, hi, base, s_, y_);
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            lo[g] = max(lo[g], qrow - wk.W + 1 - base[g]);
+            hi[g] = min(hi[g], qrow - base[g]);
+          }
+#pragma unroll
+          for (int c = 0; c < kKT; ++c) {
+            const bool ok = (c >= lo[0] && c <= hi[0]) || (c >= lo[1] && c <= hi[1]);
+            s[c] = ok ? s[c] : -INFINITY;
+          }
+        }
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < kKT; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
+        const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float m_tile = m_raw * p.scale_log2;
+        const bool grow = m_tile > m_run + kLazyRescaleLog2;
+        const float m_new = grow ? m_tile : m_run;
+        const float alpha = grow ? ex2(m_run - m_new) : 1.f;
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        float sm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < kKT; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s[c + i] = ex2(fmaf(s[c + i], p.scale_log2, -m_use));
+            sm[i] += s[c + i];
+          }
+        const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+        l_run = l_run * alpha + rs;
+        m_run = m_new;
+        // P (bf16 pairs, key 2c in the low half of column c) over the first 64 columns of S_X
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[h2 * 64 + 2 * i], s[h2 * 64 + 2 * i + 1]);
+          tmem_st32(tS + h2 * 32, pk);
+        }
+        // O_X is stable: PV_X of the previous tile was issued before this S_X
+        if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int cb2 = 0; cb2 < D / 32; ++cb2) {
+            uint32_t o32[32];
+            tmem_ld32(tO + cb2 * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+            tmem_st32(tO + cb2 * 32, o32);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR_P + 8 * x);
+        ++nt;
+      }
+      // every PV of this unit is done
+      mbar_wait(BAR_O + 8 * x, u_iter & 1, abort_flag);
+      ++u_iter;
+      tc_fence_after();
+      if (nt > 0) {
+        const float inv_l = 1.f / l_run;
+        const int hh = U.h[x];
+        __nv_bfloat16 *orow =
+            p.out + (static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow) * static_cast<int64_t>(D);
+#pragma unroll
+        for (int cb2 = 0; cb2 < D / 32; ++cb2) {
+          uint32_t o32[32];
+          tmem_ld32(tO + cb2 * 32, o32);
+          if (qrow < p.n_q) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(o32[i + 0]) * inv_l, __uint_as_float(o32[i + 1]) * inv_l);
+              v.y = pack_bf16(__uint_as_float(o32[i + 2]) * inv_l, __uint_as_float(o32[i + 3]) * inv_l);
+              v.z = pack_bf16(__uint_as_float(o32[i + 4]) * inv_l, __uint_as_float(o32[i + 5]) * inv_l);
+              v.w = pack_bf16(__uint_as_float(o32[i + 6]) * inv_l, __uint_as_float(o32[i + 7]) * inv_l);
+              *reinterpret_cast<uint4 *>(orow + cb2 * 32 + i) = v;
+            }
+          }
+        }
+        if (p.lse && qrow < p.n_q)
+          p.lse[static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow] =
+              (m_run + __log2f(l_run)) * 0.6931471805599453f;
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace swa

@@ -16,14 +16,14 @@
 #include "../../include/swa.h"
 #include "sm100.cuh"
 #include "swa_decode.cuh"
-#include "swa_fwd.cuh"
+#include "swa_fwd2.cuh"
 #include "swa_meta.cuh"
 #include "swa_tile.cuh"
 
 namespace {
 
-using swa::kBK;
-using swa::kBQ;
+constexpr int kBQ = swa::kQT;
+constexpr int kBK = swa::kKT;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -80,17 +80,25 @@ int common_checks(int B, int H, int Hkv, int d, int64_t W, float scale) {
 
 template <int D, int MODE>
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-               const CUtensorMap &tkr, const CUtensorMap &tvr, const swa::FwdParams &p,
+               const CUtensorMap &tkr, const CUtensorMap &tvr, swa::Fwd2Params p,
                cudaStream_t st) {
-  using L = swa::FwdLayout<D>;
-  auto kern = swa::fwd_kernel<D, MODE>;
+  using L = swa::Fwd2Layout<D>;
+  auto kern = swa::fwd2_kernel<D, MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
       cudaSuccess)
     return SWA_ERR_CUDA;
-  const int64_t blocks = static_cast<int64_t>(p.nqt) * p.B * p.H;
-  if (blocks > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(blocks), swa::kFwdThreads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr,
-                                                                          p);
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  const int64_t units = p.pair_heads
+                            ? static_cast<int64_t>(p.B) * p.Hkv * (p.G / 2) * p.nqt
+                            : static_cast<int64_t>(p.B) * p.H * ((p.nqt + 1) / 2);
+  if (units > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(units);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return SWA_ERR_CUDA;
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  kern<<<grid, swa::kFwd2Threads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr, p);
   return check_launch();
 }
 
@@ -181,12 +189,12 @@ int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
   if (e) return e;
   if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
-  if (N < 1 || N >= (int64_t(1) << 30)) return SWA_ERR_INVALID_ARG;
+  if (N < 1 || N >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv;
   if ((e = make_map(&tq, q, d, N, static_cast<int64_t>(B) * H, kBQ))) return e;
   if ((e = make_map(&tk, k, d, N, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tv, v, d, N, static_cast<int64_t>(B) * Hkv, kBK))) return e;
-  swa::FwdParams p;
+  swa::Fwd2Params p;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
   p.q_start = nullptr;
@@ -234,14 +242,14 @@ int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, voi
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
       !aligned16(v_ring) || !aligned16(out))
     return SWA_ERR_INVALID_ARG;
-  if (Tq < 1 || Tq >= (int64_t(1) << 30) || W >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  if (Tq < 1 || Tq >= (int64_t(1) << 29) || W >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv, tkr, tvr;
   if ((e = make_map(&tq, q, d, Tq, static_cast<int64_t>(B) * H, kBQ))) return e;
   if ((e = make_map(&tk, k_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tv, v_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tkr, k_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tvr, v_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
-  swa::FwdParams p;
+  swa::Fwd2Params p;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
   p.q_start = q_start;
