@@ -85,6 +85,15 @@ def algorithmic_bytes(w) -> int:
 
 # ----------------------------------------------------------------------------- helpers
 
+def describe(w) -> str:
+    if w.kind == "prefill":
+        return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} N{w.N} d{w.d} W{w.W}"
+    if w.kind == "chunk":
+        return (f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} Tq{w.Tq} d{w.d} W{w.W} "
+                f"q_start{w.q_start}")
+    return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} d{w.d} W{w.W} ctx U[{w.ctx_lo},{w.ctx_hi}]"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -95,13 +104,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "fwd2_kernel": ("swa_fwd2.cuh", "swa_tile.cuh", "sm100.cuh"),
+    "decode_split_kernel": ("swa_decode.cuh", "sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """sha256 (16 hex) of the source files a kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sliding_window_sparse_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -114,7 +129,7 @@ def profiled_traffic(kernel: str, workload: str):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
     s = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_hash():
+    if not m or not s or s.group(1) != kernel_source_hash(kernel):
         return None
     return int(m.group(1))
 
@@ -133,7 +148,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", gpu_id, "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                 "-i", gpu_id, "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                 text=True)
         except OSError:
             return
@@ -394,8 +409,9 @@ def run_native(args):
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
     sampler = ClockSampler(gpu_id) if rank == 0 else None
 
-    # headline: the Mistral-shaped prefill, each rank its own batch
-    w = WORKLOADS[HEADLINE]
+    # headline (default: the Mistral-shaped prefill), each rank its own batch
+    headline = args.workload
+    w = WORKLOADS[headline]
     x = make_inputs(w, dev, seed_offset=rank)
     call, out, launches_per_step = make_call(w, x, swa)
     times, t0, t1 = time_steps(call, args.steps, args.warmup, flush, barrier)
@@ -403,21 +419,26 @@ def run_native(args):
         raise SystemExit("device status error during the timed region")
     total_ms = max_over_ranks(sum(times))
     mean_ms = total_ms / args.steps
-    flops = useful_flops(w)
-    value = flops * world / (mean_ms * 1e-3) / 1e12
-    kernel_tflops = flops / (statistics.mean(times) * 1e-3) / 1e12
+    if w.kind == "decode":
+        work, unit, scale_div, bound, peak = decode_kv_bytes(w), "GB/s", 1e9, "hbm", "hbm_gbs"
+    else:
+        work, unit, scale_div, bound, peak = useful_flops(w), "TFLOP/s", 1e12, "tensor", "bf16_tflops"
+    value = work * world / (mean_ms * 1e-3) / scale_div
+    kernel_rate = work / (statistics.mean(times) * 1e-3) / scale_div
     clocks = sampler.summary(t0, t1) if sampler else None
 
     # end to end through the public API with host buffers
     e2e_steps = max(3, min(args.steps, 20))
     e2e_ms, h2d, d2h = time_e2e(w, x, swa, e2e_steps, 2)
     e2e_ms = max_over_ranks(e2e_ms)
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = work * world / (e2e_ms * 1e-3) / scale_div
 
     # the other paths of the hot path, on their own workloads
     paths = {}
     if not args.headline_only:
-        for name in ("narrow_window", "chunk_ring", "decode_ring"):
+        for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring"):
+            if name == headline:
+                continue
             pw = WORKLOADS[name]
             px = make_inputs(pw, dev, seed_offset=rank)
             pcall, _, nl = make_call(pw, px, swa)
@@ -447,31 +468,33 @@ def run_native(args):
 
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and w.kind == "prefill":
             import oracle
 
             host = host_prefill_inputs(x)
             dt, fl, n_rows = calibrated_oracle(w, host, args.cpu_seconds)
             cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                    "kind": "oracle",
-                   "sample": f"{n_rows} random query rows of {HEADLINE} (full window each), "
+                   "sample": f"{n_rows} random query rows of {headline} (full window each), "
                              f"{dt:.1f} s"}
-        roof = {"bound": "tensor", "achieved": kernel_tflops, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": kernel_tflops / peaks["bf16_tflops"],
-                "traffic": profiled_traffic("fwd_kernel", HEADLINE),
-                "peak_source": f"{peak_src} bf16 burst",
-                "frac_of_sustained": kernel_tflops / peaks["bf16_tflops_sustained"],
+        kname = "decode_split_kernel" if w.kind == "decode" else "fwd2_kernel"
+        roof = {"bound": bound, "achieved": kernel_rate, "peak": peaks[peak], "unit": unit,
+                "frac": kernel_rate / peaks[peak],
+                "traffic": profiled_traffic(kname, headline),
+                "peak_source": f"{peak_src} " + ("bf16 burst" if bound == "tensor" else "copy"),
                 "algorithmic_bytes": algorithmic_bytes(w)}
+        if bound == "tensor":
+            roof["frac_of_sustained"] = kernel_rate / peaks["bf16_tflops_sustained"]
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{HEADLINE}: B1 H32 Hkv8 N8192 d128 W4096 (one batch per rank)",
-                       "useful_flops_per_step": flops, "l2": "flushed by a 256 MiB write "
+            "config": {"workload": describe(w) + " (one batch per rank)",
+                       "work_per_step": work, "l2": "flushed by a 256 MiB write "
                        "between timed steps"},
             "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks, "paths": paths,
@@ -485,12 +508,14 @@ def run_native(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE,
+                    help="headline workload (default: the Mistral-shaped prefill)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
