@@ -170,6 +170,27 @@ SWA_API int swa_attn_decode_ring(const void *q, const void *k_ring, const void *
                          size_t workspace_bytes, void *stream);
 
 /*
+ * swa_attn_decode_ring_static -- swa_attn_decode_ring without a workspace.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device scratch (a plugin or foreign-language host with
+ * no device allocator, or a process that reserved all free device memory up
+ * front).  Same arguments, layouts and results as swa_attn_decode_ring; the
+ * split partials live in a fixed 16 MiB (16777216-byte) device array that
+ * every device loading the library keeps until exit.  Calls no allocator.
+ *  - Returns SWA_ERR_WORKSPACE, before enqueuing anything, when
+ *    swa_decode_workspace_bytes(B, H, Hkv, d, W) exceeds 16777216 bytes.
+ *  - All calls on a device share the array (it keeps the last call's
+ *    contents; nothing needs to start zeroed): calls whose kernels overlap on
+ *    one device race and must be ordered on one stream or with events.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress with that device current) and caches it; make
+ *    that first call before any stream capture.
+ */
+SWA_API int swa_attn_decode_ring_static(const void *q, const void *k_ring, const void *v_ring,
+                                        const int64_t *pos, void *out, float *lse, int B, int H,
+                                        int Hkv, int d, int64_t W, float scale, void *stream);
+
+/*
  * swa_ring_slot_positions -- the logical position held by every ring slot.
  * Passage: M003 note section 06 (logical vs physical slots); blog section 3.2.
  * For sequence b after positions 0 .. n_written[b]-1 were written:

@@ -29,6 +29,7 @@ __all__ = [
     "swa_ring_write",
     "swa_decode_workspace_bytes",
     "swa_attn_decode_ring",
+    "swa_attn_decode_ring_static",
     "swa_ring_slot_positions",
     "swa_get_device_status",
     "swa_version",
@@ -170,6 +171,37 @@ def swa_attn_decode_ring(q, k_ring, v_ring, pos, scale: float | None = None, wor
                                      _ptr(lse), B, H, Hkv, d, W, scale, _ptr(workspace),
                                      workspace.numel() * workspace.element_size(),
                                      _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_attn_decode_ring_static(q, k_ring, v_ring, pos, scale: float | None = None, out=None,
+                                lse=None, return_lse: bool = False):
+    """Decode like swa_attn_decode_ring, for callers that cannot provide device scratch.
+
+    The library keeps the split partials in its own fixed 16 MiB device array,
+    so nothing is allocated for scratch; larger requests raise SwaError
+    (SWA_ERR_WORKSPACE).
+    Calls on one device share that array: do not let two of them overlap on
+    the GPU (keep them on one stream or order them with events).  The first
+    call on a device resolves the array's address; make it before any stream
+    capture.
+    """
+    _need(q, "q", dims=3)
+    _need(k_ring, "k_ring", dims=4)
+    _need(v_ring, "v_ring", dims=4)
+    _need(pos, "pos", torch.int64, 1)
+    B, H, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    check("swa_attn_decode_ring_static",
+          lib().swa_attn_decode_ring_static(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(pos),
+                                            _ptr(out), _ptr(lse), B, H, Hkv, d, W, scale,
+                                            _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

@@ -31,6 +31,7 @@ SIGNATURES = {
     "swa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i64]),
     "swa_attn_decode_ring": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i64, _f, _p, _sz, _p]),
     "swa_ring_slot_positions": (_i, [_i, _p, _i64, _p, _p]),
+    "swa_attn_decode_ring_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i64, _f, _p]),
     "swa_get_device_status": (_i, [_p]),
 }
 

@@ -335,3 +335,77 @@ int swa_get_device_status(void *stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers have no way to give this library device scratch: a plugin or a
+// foreign-language host that owns no device allocator of its own, or a
+// serving process that reserved all free device memory for its KV cache up
+// front and forbids later allocations.  For them swa_attn_decode_ring_static
+// runs the same split and merge kernels as swa_attn_decode_ring, with the
+// split partials kept in the file-scope device array below instead of a
+// workspace argument.  It calls no allocator (cudaMalloc, cudaFree or any
+// library routine that allocates).
+//
+// The array is g_swa_static_scratch_bytes (16 MiB) long on every device that loads
+// this library and stays resident until the process exits.  All calls on a
+// device share it and it keeps the last call's contents; nothing in it has to
+// start at zero, because every split partial is written before the merge
+// reads it.  Two calls whose kernels overlap on the same device (for example
+// on two streams without ordering between them) race on the array and give
+// wrong results: order such calls on one stream or with events.
+//
+// Host code cannot use the array's name as a device address, so the first
+// call on each device looks the address up with cudaGetSymbolAddress while
+// that device is current and caches it; make that first call before any
+// stream capture.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t g_swa_static_scratch_bytes = size_t(16) << 20;  // 16 MiB per device
+static __device__ __align__(256) unsigned char g_swa_static_scratch[g_swa_static_scratch_bytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mutex;
+void *g_static_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device (looked up once per device).
+int static_scratch_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SWA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SWA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_swa_static_scratch) != cudaSuccess || !ptr)
+      return SWA_ERR_CUDA;
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return SWA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int swa_attn_decode_ring_static(const void *q, const void *k_ring, const void *v_ring,
+                                const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
+                                int d, int64_t W, float scale, void *stream) {
+  int e = common_checks(B, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k_ring || !v_ring || !pos || !out) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out))
+    return SWA_ERR_INVALID_ARG;
+  if (W >= (int64_t(1) << 31) || B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+  // the split partials must fit in the static array
+  const size_t need = swa_decode_workspace_bytes(B, H, Hkv, d, W);
+  if (need == 0 || need > g_swa_static_scratch_bytes) return SWA_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  if ((e = static_scratch_address(&scratch))) return e;
+  return swa_attn_decode_ring(q, k_ring, v_ring, pos, out, lse, B, H, Hkv, d, W, scale, scratch,
+                              g_swa_static_scratch_bytes, stream);
+}
+
+}  // extern "C"
