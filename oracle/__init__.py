@@ -63,32 +63,60 @@ def _load():
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB)
-            lib.orc_num_threads.restype = _int
-            lib.orc_count_pairs.restype = _i64
-            lib.orc_count_pairs.argtypes = [_i64, _i64]
-            lib.orc_swa_forward.restype = _i64
-            lib.orc_swa_forward.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
-                                            _dbl, _ptr, _ptr, _i64, _ptr, _ptr]
-            lib.orc_dense_masked.restype = _int
-            lib.orc_dense_masked.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
-                                             _dbl, _ptr]
-            lib.orc_ring_positions.restype = None
-            lib.orc_ring_positions.argtypes = [_i64, _i64, _ptr]
-            lib.orc_swa_chunk.restype = _i64
-            lib.orc_swa_chunk.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int,
-                                          _i64, _int, _i64, _dbl, _ptr, _i64, _ptr, _ptr]
-            lib.orc_ring_update.restype = None
-            lib.orc_ring_update.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _i64, _int,
-                                            _i64]
-            lib.orc_swa_decode.restype = _i64
-            lib.orc_swa_decode.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int, _i64,
-                                           _dbl, _ptr, _ptr]
-            lib.orc_tile_classes.restype = _int
-            lib.orc_tile_classes.argtypes = [_int, _int, _i64, _i64, _ptr, _i64, _int, _int, _ptr,
-                                             _ptr]
+            lib = _configure(ctypes.CDLL(_LIB))
             _lib = lib
     return _lib
+
+
+def _configure(lib):
+    """Declare the C signatures on a loaded build of swa_oracle.c."""
+    lib.orc_num_threads.restype = _int
+    lib.orc_count_pairs.restype = _i64
+    lib.orc_count_pairs.argtypes = [_i64, _i64]
+    lib.orc_swa_forward.restype = _i64
+    lib.orc_swa_forward.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
+                                    _dbl, _ptr, _ptr, _i64, _ptr, _ptr]
+    lib.orc_dense_masked.restype = _int
+    lib.orc_dense_masked.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
+                                     _dbl, _ptr]
+    lib.orc_ring_positions.restype = None
+    lib.orc_ring_positions.argtypes = [_i64, _i64, _ptr]
+    lib.orc_swa_chunk.restype = _i64
+    lib.orc_swa_chunk.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int,
+                                  _i64, _int, _i64, _dbl, _ptr, _i64, _ptr, _ptr]
+    lib.orc_ring_update.restype = None
+    lib.orc_ring_update.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _i64, _int,
+                                    _i64]
+    lib.orc_swa_decode.restype = _i64
+    lib.orc_swa_decode.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int, _i64,
+                                   _dbl, _ptr, _ptr]
+    lib.orc_tile_classes.restype = _int
+    lib.orc_tile_classes.argtypes = [_int, _int, _i64, _i64, _ptr, _i64, _int, _int, _ptr,
+                                     _ptr]
+    return lib
+
+
+class use_library:
+    """Context manager (tests only): route every oracle call to another build of
+    swa_oracle.c, e.g. a copy with a planted mistake, then restore."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _lib
+        _load()
+        with _lock:
+            self.saved = _lib
+            _lib = _configure(ctypes.CDLL(self.path))
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self.saved
+        return False
 
 
 def _p(a):
