@@ -207,6 +207,37 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Bits a..b (inclusive, clipped to 0..31) of a 32-bit word; 0 if the range is empty.
+__device__ __forceinline__ uint32_t range_bits(int a, int b) {
+  if (b < 0 || a > 31 || a > b) return 0u;
+  a = a < 0 ? 0 : a;
+  b = b > 31 ? 31 : b;
+  return (0xFFFFFFFFu >> (31 - (b - a))) << a;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe for a pair of values, x >= -125 (finite).
+// Range reduction x = n + f, n = round(x) (added to the exponent field),
+// f in [-1/2, 1/2]; 2^f from a degree-3 minimax polynomial for the relative
+// error (coefficients fitted by fit_exp2_poly.py: max relative error 7.5e-5).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const float2 t = __fadd2_rn(x, magic);                      // n in the low mantissa bits
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __fadd2_rn(x, make_float2(-r.x, -r.y));
+  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

@@ -9,10 +9,10 @@
 // units c, c + gridDim.x, ... (heavy query tiles first).
 //
 // Roles (320 threads):
-//   warp 0      TMA producer: Q_A, Q_B once per unit, then K/V tiles into a
-//               2-stage shared-memory ring (128-byte swizzle, one box per 64
-//               head-dim columns).  Only live key tiles are loaded (M003 note
-//               section 04).
+//   warp 0      TMA producer: Q_A, Q_B once per unit, then K and V tiles into
+//               separate shared-memory rings (3 K and 2 V stages at d = 128;
+//               128-byte swizzle, one box per 64 head-dim columns).  Only live
+//               key tiles are loaded (M003 note section 04).
 //   warp 1      one thread issues every tcgen05.mma:
 //                 S_X = Q_X K^T        (A, B from shared memory)
 //                 O_X += P_X V         (P from tensor memory, V from shared memory)
@@ -45,6 +45,13 @@ constexpr int kQT = 128;  // query rows per tile (MMA M, tensor-memory lanes)
 constexpr int kKT = 128;  // keys per tile
 constexpr int kFwd2Threads = 320;
 constexpr float kLazyRescaleLog2 = 8.0f;
+// The exponentials of the last kEmuCols columns of every tile are evaluated
+// on the FMA pipe (ex2_poly2) instead of the MUFU, to balance the two pipes.
+#ifndef SWA_EMU_COLS
+#define SWA_EMU_COLS 0
+#endif
+constexpr int kEmuCols = SWA_EMU_COLS;
+static_assert(kEmuCols % 16 == 0 && kEmuCols <= 128, "emulated columns in groups of 16");
 
 struct Fwd2Params {
   __nv_bfloat16 *out;      // [B, H, n_q, D]
@@ -64,16 +71,20 @@ struct Fwd2Params {
 template <int D>
 struct Fwd2Layout {
   static constexpr int PANELS = D / 64;
-  static constexpr int NST = D == 64 ? 4 : 2;
+  // K and V have rings of their own: a K tile is free once both S MMAs have
+  // read it, a V tile once both PV MMAs have, so K is released one step early.
+  static constexpr int NK = D == 64 ? 4 : 3;  // K stages
+  static constexpr int NV = D == 64 ? 4 : 2;  // V stages
   static constexpr uint32_t Q_BYTES = kQT * D * 2;
   static constexpr uint32_t KV_BYTES = kKT * D * 2;
   static constexpr uint32_t OFF_QA = 0;
   static constexpr uint32_t OFF_QB = Q_BYTES;
   static constexpr uint32_t OFF_K = 2 * Q_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + NST * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + NST * KV_BYTES;
-  // q_full, q_empty, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2], o_full[2]
-  static constexpr int NBAR = 2 + 3 * NST + 6;
+  static constexpr uint32_t OFF_V = OFF_K + NK * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NV * KV_BYTES;
+  // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
+  // o_full[2]
+  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 6;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t BYTES = OFF_MISC + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;
@@ -223,7 +234,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_vr, const Fwd2Params p) {
   using L = Fwd2Layout<D>;
-  constexpr int NST = L::NST;
+  constexpr int NK = L::NK, NV = L::NV;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -231,10 +242,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
   const uint32_t sQ[2] = {base + L::OFF_QA, base + L::OFF_QB};
   const uint32_t sK = base + L::OFF_K, sV = base + L::OFF_V, bar = base + L::OFF_BAR;
   const uint32_t BAR_QF = bar, BAR_QE = bar + 8;
-  const uint32_t BAR_KF = bar + 16;                 // + 8 * stage
-  const uint32_t BAR_VF = bar + 16 + 8 * NST;       // + 8 * stage
-  const uint32_t BAR_KVE = bar + 16 + 16 * NST;     // + 8 * stage
-  const uint32_t BAR_S = bar + 16 + 24 * NST;       // + 8 * tile
+  const uint32_t BAR_KF = bar + 16;                 // + 8 * K stage
+  const uint32_t BAR_KE = BAR_KF + 8 * NK;          // + 8 * K stage
+  const uint32_t BAR_VF = BAR_KE + 8 * NK;          // + 8 * V stage
+  const uint32_t BAR_VE = BAR_VF + 8 * NV;          // + 8 * V stage
+  const uint32_t BAR_S = BAR_VE + 8 * NV;           // + 8 * tile
   const uint32_t BAR_P = BAR_S + 16;                // + 8 * tile
   const uint32_t BAR_O = BAR_P + 16;                // + 8 * tile
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
@@ -244,10 +256,13 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
   if (threadIdx.x == 0) {
     mbar_init(BAR_QF, 1);
     mbar_init(BAR_QE, 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(BAR_KF + 8 * s, 1);
+      mbar_init(BAR_KE + 8 * s, 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(BAR_VF + 8 * s, 1);
-      mbar_init(BAR_KVE + 8 * s, 1);
+      mbar_init(BAR_VE + 8 * s, 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(BAR_S + 8 * x, 1);
@@ -311,20 +326,22 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         int k, src, y0, ca, cb;
         const int z = U.b * p.Hkv + U.kvh;
         while (wk.next(k, src, y0, ca, cb)) {
-          const int st = kv_iter % NST;
-          if (kv_iter >= NST && !mbar_wait(BAR_KVE + 8 * st, ((kv_iter / NST) - 1) & 1, abort_flag))
-            break;
+          const int sk = kv_iter % NK, sv = kv_iter % NV;
           const CUtensorMap *mk = src == 1 ? &tm_kr : &tm_k;
           const CUtensorMap *mv = src == 1 ? &tm_vr : &tm_v;
-          mbar_expect_tx(BAR_KF + 8 * st, L::KV_BYTES);
+          if (kv_iter >= NK && !mbar_wait(BAR_KE + 8 * sk, ((kv_iter / NK) - 1) & 1, abort_flag))
+            break;
+          mbar_expect_tx(BAR_KF + 8 * sk, L::KV_BYTES);
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
-            tma_load_3d(sK + st * L::KV_BYTES + pn * (kKT * 128), mk, BAR_KF + 8 * st, pn * 64,
+            tma_load_3d(sK + sk * L::KV_BYTES + pn * (kKT * 128), mk, BAR_KF + 8 * sk, pn * 64,
                         y0, z);
-          mbar_expect_tx(BAR_VF + 8 * st, L::KV_BYTES);
+          if (kv_iter >= NV && !mbar_wait(BAR_VE + 8 * sv, ((kv_iter / NV) - 1) & 1, abort_flag))
+            break;
+          mbar_expect_tx(BAR_VF + 8 * sv, L::KV_BYTES);
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
-            tma_load_3d(sV + st * L::KV_BYTES + pn * (kKT * 128), mv, BAR_VF + 8 * st, pn * 64,
+            tma_load_3d(sV + sv * L::KV_BYTES + pn * (kKT * 128), mv, BAR_VF + 8 * sv, pn * 64,
                         y0, z);
           ++kv_iter;
         }
@@ -369,11 +386,12 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         bool have = wk.next(k, src, y0, ca, cb);
         bool first[2] = {true, true};
         if (have) {
-          const int st = kv_iter % NST;
-          mbar_wait(BAR_KF + 8 * st, (kv_iter / NST) & 1, abort_flag);
+          const int sk = kv_iter % NK;
+          mbar_wait(BAR_KF + 8 * sk, (kv_iter / NK) & 1, abort_flag);
           tc_fence_after();
-          if (ca) issue_s(0, st);
-          if (cb) issue_s(1, st);
+          if (ca) issue_s(0, sk);
+          if (cb) issue_s(1, sk);
+          tc_commit(BAR_KE + 8 * sk);  // K(first) is read by both S MMAs
         } else {
           tc_commit(BAR_QE);
         }
@@ -381,27 +399,33 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           int na = 0, nb = 0;
           const bool has_next = wk.next(k, src, y0, na, nb);
           if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
-          const int st = kv_iter % NST;
-          const int stn = (kv_iter + 1) % NST;
-          mbar_wait(BAR_VF + 8 * st, (kv_iter / NST) & 1, abort_flag);
-          if (has_next) mbar_wait(BAR_KF + 8 * stn, ((kv_iter + 1) / NST) & 1, abort_flag);
+          const int sv = kv_iter % NV;
+          const int skn = (kv_iter + 1) % NK;
+          mbar_wait(BAR_VF + 8 * sv, (kv_iter / NV) & 1, abort_flag);
           if (ca) {
             mbar_wait(BAR_P, p_cnt[0] & 1, abort_flag);
             ++p_cnt[0];
             tc_fence_after();
-            issue_pv(0, st, !first[0]);
+            issue_pv(0, sv, !first[0]);
             first[0] = false;
           }
-          if (has_next && na) issue_s(0, stn);
+          if (has_next) {
+            mbar_wait(BAR_KF + 8 * skn, ((kv_iter + 1) / NK) & 1, abort_flag);
+            tc_fence_after();
+            if (na) issue_s(0, skn);
+          }
           if (cb) {
             mbar_wait(BAR_P + 8, p_cnt[1] & 1, abort_flag);
             ++p_cnt[1];
             tc_fence_after();
-            issue_pv(1, st, !first[1]);
+            issue_pv(1, sv, !first[1]);
             first[1] = false;
           }
-          if (has_next && nb) issue_s(1, stn);
-          tc_commit(BAR_KVE + 8 * st);
+          tc_commit(BAR_VE + 8 * sv);  // V(j) is read by both PV MMAs
+          if (has_next) {
+            if (nb) issue_s(1, skn);
+            tc_commit(BAR_KE + 8 * skn);
+          }
           ++kv_iter;
           ca = na;
           cb = nb;
@@ -441,7 +465,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         tmem_ld128(tS, sr);
         float *s = reinterpret_cast<float *>(sr);
         if (cls == 2) {
-          // allowed columns of this row: c in a segment with base + c in [q - W + 1, q]
+          // allowed columns of this row: c in a segment with base + c in [q - W + 1, q],
+          // as a 128-bit mask (one word per 32 columns)
           int lo[2], hi[2], base[2], s_, y_;
           wk.segments(k, lo, hi, base, s_, y_);
 #pragma unroll
@@ -449,37 +474,54 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             lo[g] = max(lo[g], qrow - wk.W + 1 - base[g]);
             hi[g] = min(hi[g], qrow - base[g]);
           }
+          uint32_t mw[kKT / 32];
 #pragma unroll
-          for (int c = 0; c < kKT; ++c) {
-            const bool ok = (c >= lo[0] && c <= hi[0]) || (c >= lo[1] && c <= hi[1]);
-            s[c] = ok ? s[c] : -INFINITY;
-          }
+          for (int w = 0; w < kKT / 32; ++w)
+            mw[w] = range_bits(lo[0] - 32 * w, hi[0] - 32 * w) |
+                    range_bits(lo[1] - 32 * w, hi[1] - 32 * w);
+#pragma unroll
+          for (int c = 0; c < kKT; ++c) s[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
         }
         float mx[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx[i] = s[i];
 #pragma unroll
-        for (int c = 8; c < kKT; c += 8)
+        for (int c = 8; c + 16 <= kKT; c += 16)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
-        const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[kKT - 8 + i]);
+        const float m_raw = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
         const float m_tile = m_raw * p.scale_log2;
         const bool grow = m_tile > m_run + kLazyRescaleLog2;
         const float m_new = grow ? m_tile : m_run;
         const float alpha = grow ? ex2(m_run - m_new) : 1.f;
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        float sm[8];
+        // x = s * scale * log2(e) - m, two columns per packed FMA
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_use, -m_use);
+        float2 *s2 = reinterpret_cast<float2 *>(s);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+        for (int c = 0; c < kKT / 2; ++c) s2[c] = __ffma2_rn(s2[c], sc2, nm2);
+        // exponentials: MUFU for the first columns, FMA-pipe polynomial for the last
+        // kEmuCols (a masked column clamps to 2^-125 there, which is numerically 0
+        // next to the row maximum's 2^0 and is cleared with O and l by any later
+        // rescale)
 #pragma unroll
-        for (int c = 0; c < kKT; c += 8)
+        for (int c = 0; c < kKT - kEmuCols; ++c) s[c] = ex2(s[c]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            s[c + i] = ex2(fmaf(s[c + i], p.scale_log2, -m_use));
-            sm[i] += s[c + i];
-          }
-        const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+        for (int c = (kKT - kEmuCols) / 2; c < kKT / 2; ++c)
+          s2[c] = ex2_poly2(make_float2(fmaxf(s2[c].x, -125.f), fmaxf(s2[c].y, -125.f)));
+        float2 sm2[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kKT / 2; c += 4)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sm2[i] = __fadd2_rn(sm2[i], s2[c + i]);
+        const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
+        const float rs = sa.x + sa.y;
         l_run = l_run * alpha + rs;
         m_run = m_new;
         // P (bf16 pairs, key 2c in the low half of column c) over the first 64 columns of S_X
