@@ -138,6 +138,7 @@ struct Walker2 {
   int wrap;      // MODE 1: ring full ? L mod W : number of filled slots
   bool full_ring;
   bool has_b;
+  int live_a_end, live_b_begin;  // MODE 0: A is live on [kt, live_a_end], B on [live_b_begin, kt_end)
 
   __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs) {
     has_b = U.has_b;
@@ -151,6 +152,10 @@ struct Walker2 {
     if (MODE == 0) {
       kt = max(qlo[0] - (W - 1), 0) / kKT;
       kt_end = (has_b ? qhi[1] : qhi[0]) / kKT + 1;
+      // the windows of consecutive rows overlap, so each tile's live key tiles are
+      // one contiguous range: [first key of its first row, its last row] in tiles
+      live_a_end = qhi[0] / kKT;
+      live_b_begin = max(qlo[1] - (W - 1), 0) / kKT;
       nrt = 0;
       wrap = 0;
       full_ring = false;
@@ -212,6 +217,22 @@ struct Walker2 {
     // A ragged tile (nc < kKT) is masked even when every in-range pair is allowed:
     // its out-of-range columns read as zero and must not enter the softmax.
     return !any ? 0 : (all_cols == nc && nc == kKT ? 1 : 2);
+  }
+
+  // Advance to the next live tile, reporting only which query tiles use it
+  // (ca, cb nonzero) -- what the producer and the MMA issuer need.  MODE 0
+  // reduces to two comparisons per tile; MODE 1 runs the full classification.
+  __device__ __forceinline__ bool next_live(int &k, int &src, int &y0, int &ca, int &cb) {
+    if (MODE == 0) {
+      if (kt >= kt_end) return false;
+      k = kt++;
+      src = 0;
+      y0 = k * kKT;
+      ca = k <= live_a_end;
+      cb = has_b && k >= live_b_begin;
+      return true;
+    }
+    return next(k, src, y0, ca, cb);
   }
 
   // Advance to the next live tile: its index, source, first row and classes.
@@ -325,7 +346,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         wk.init(U, p, qs);
         int k, src, y0, ca, cb;
         const int z = U.b * p.Hkv + U.kvh;
-        while (wk.next(k, src, y0, ca, cb)) {
+        while (wk.next_live(k, src, y0, ca, cb)) {
           const int sk = kv_iter % NK, sv = kv_iter % NV;
           const CUtensorMap *mk = src == 1 ? &tm_kr : &tm_k;
           const CUtensorMap *mv = src == 1 ? &tm_vr : &tm_v;
@@ -383,7 +404,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         Walker2<MODE> wk;
         wk.init(U, p, qs);
         int k, src, y0, ca, cb;
-        bool have = wk.next(k, src, y0, ca, cb);
+        bool have = wk.next_live(k, src, y0, ca, cb);
         bool first[2] = {true, true};
         if (have) {
           const int sk = kv_iter % NK;
@@ -397,7 +418,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         }
         while (have) {
           int na = 0, nb = 0;
-          const bool has_next = wk.next(k, src, y0, na, nb);
+          const bool has_next = wk.next_live(k, src, y0, na, nb);
           if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
           const int sv = kv_iter % NV;
           const int skn = (kv_iter + 1) % NK;
