@@ -5,8 +5,8 @@
 // tiles.  With G = H / Hkv even they are two query heads of one key/value
 // group at the same query rows (identical tile lists); otherwise they are
 // query tiles 2p and 2p+1 of one head (the key stream is the union of both
-// windows and each tile uses its own part).  CTAs are persistent: CTA c takes
-// units c, c + gridDim.x, ... (heavy query tiles first).
+// windows and each tile uses its own part).  CTAs are persistent and walk the
+// heavy-first unit order in a serpentine (see unit_of).
 //
 // Roles (320 threads):
 //   warp 0      TMA producer: Q_A, Q_B once per unit, then K and V tiles into
@@ -311,6 +311,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Serpentine static schedule over the heavy-first unit order: in round r
+  // CTA c takes unit r * P + c (r even) or r * P + P - 1 - c (r odd), which
+  // pairs heavy with light units.
+  auto unit_of = [&](int i) -> int {
+    const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return i * P + ((i & 1) ? P - 1 - c : c);
+  };
+
   auto unit_start = [&](const Unit &U, int64_t &qs) -> bool {
     qs = 0;
     if (MODE == 1) {
@@ -324,7 +332,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int kv_iter = 0, q_iter = 0;
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         const Unit U = decode_unit(u, p);
         int64_t qs;
         if (!unit_start(U, qs)) {
@@ -395,7 +403,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           mma_ts(dO, aP + kk * 8, sdesc_sw128(sV + st * L::KV_BYTES + kk * 16 * 128, kKT * 128, 1024),
                  idO, (acc || kk > 0) ? 1u : 0u);
       };
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         const Unit U = decode_unit(u, p);
         int64_t qs;
         if (!unit_start(U, qs)) continue;
@@ -403,22 +411,37 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         tc_fence_after();
         Walker2<MODE> wk;
         wk.init(U, p, qs);
-        int k, src, y0, ca, cb;
+        int k, src, y0, ca, cb, na = 0, nb = 0;
         bool have = wk.next_live(k, src, y0, ca, cb);
         bool first[2] = {true, true};
-        if (have) {
+        if (!have) {  // (no live tile: keep every barrier's phase count in step)
+          tc_commit(BAR_QE);
+          tc_commit(BAR_O);
+          tc_commit(BAR_O + 8);
+          ++q_iter;
+          continue;
+        }
+        bool has_next = wk.next_live(k, src, y0, na, nb);
+        {
           const int sk = kv_iter % NK;
           mbar_wait(BAR_KF + 8 * sk, (kv_iter / NK) & 1, abort_flag);
           tc_fence_after();
           if (ca) issue_s(0, sk);
           if (cb) issue_s(1, sk);
-          tc_commit(BAR_KE + 8 * sk);  // K(first) is read by both S MMAs
-        } else {
-          tc_commit(BAR_QE);
         }
+        // tile B starting one tile after A (query tiles 2p, 2p+1): issue its first
+        // S now instead of behind A's first softmax
+        bool b_ahead = false;
+        if (MODE == 0 && has_next && nb && !cb) {
+          const int sk1 = (kv_iter + 1) % NK;
+          mbar_wait(BAR_KF + 8 * sk1, ((kv_iter + 1) / NK) & 1, abort_flag);
+          tc_fence_after();
+          issue_s(1, sk1);
+          b_ahead = true;
+        }
+        tc_commit(BAR_KE + 8 * (kv_iter % NK));  // K(first) is read by both S MMAs
+        bool o_done[2] = {false, false};
         while (have) {
-          int na = 0, nb = 0;
-          const bool has_next = wk.next_live(k, src, y0, na, nb);
           if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
           const int sv = kv_iter % NV;
           const int skn = (kv_iter + 1) % NK;
@@ -429,6 +452,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             tc_fence_after();
             issue_pv(0, sv, !first[0]);
             first[0] = false;
+            // linear keys: a query tile's live tiles are contiguous, so it is done
+            if (MODE == 0 && !(has_next && na)) {
+              tc_commit(BAR_O);
+              o_done[0] = true;
+            }
           }
           if (has_next) {
             mbar_wait(BAR_KF + 8 * skn, ((kv_iter + 1) / NK) & 1, abort_flag);
@@ -441,19 +469,25 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             tc_fence_after();
             issue_pv(1, sv, !first[1]);
             first[1] = false;
+            if (MODE == 0 && !(has_next && nb)) {
+              tc_commit(BAR_O + 8);
+              o_done[1] = true;
+            }
           }
           tc_commit(BAR_VE + 8 * sv);  // V(j) is read by both PV MMAs
           if (has_next) {
-            if (nb) issue_s(1, skn);
+            if (nb && !b_ahead) issue_s(1, skn);
+            b_ahead = false;
             tc_commit(BAR_KE + 8 * skn);
           }
           ++kv_iter;
           ca = na;
           cb = nb;
           have = has_next;
+          if (have) has_next = wk.next_live(k, src, y0, na, nb);
         }
-        tc_commit(BAR_O);
-        tc_commit(BAR_O + 8);
+        if (!o_done[0]) tc_commit(BAR_O);
+        if (!o_done[1]) tc_commit(BAR_O + 8);
         ++q_iter;
       }
     }
@@ -466,7 +500,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     const uint32_t tS = tmem + x * 128 + lane_off;
     const uint32_t tO = tmem + 256 + x * D + lane_off;
     uint32_t s_cnt = 0, u_iter = 0;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
       const Unit U = decode_unit(u, p);
       int64_t qs;
       if (!unit_start(U, qs)) continue;
