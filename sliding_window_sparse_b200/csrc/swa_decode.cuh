@@ -226,6 +226,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const Deco
     __syncwarp();
   }
 
+  // this CTA's loads are done: let the dependent merge kernel start launching
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // sum the partial o of the KPW key groups (same dims, different slots)
 #pragma unroll
   for (int m = LPK; m < 32; m <<= 1)
@@ -278,6 +280,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const Deco
 // Merge the split partials of one (b, h): o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
+  // launched as a programmatic dependent of the split kernel: wait for its results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t bh = blockIdx.x;
   const int c = threadIdx.x;
   const float *ml = p.ws_ml + bh * p.splits * 2;

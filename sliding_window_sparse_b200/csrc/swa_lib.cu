@@ -115,7 +115,20 @@ int launch_decode(const swa::DecodeParams &p, cudaStream_t st) {
   dim3 grid(p.splits, p.Hkv, p.B);
   swa::decode_split_kernel<D, G><<<grid, swa::kDecWarps * 32, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
-  swa::decode_combine_kernel<D><<<static_cast<unsigned>(p.B * p.H), D, 0, st>>>(p);
+  // The merge kernel is launched as a programmatic dependent of the split
+  // kernel: its CTAs may start while the last split CTAs drain and wait in
+  // griddepcontrol.wait until every split CTA's partials are visible.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.H));
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, swa::decode_combine_kernel<D>, p) != cudaSuccess) return SWA_ERR_CUDA;
   return check_launch();
 }
 
