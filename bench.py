@@ -105,7 +105,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "fwd2_kernel": ("swa_fwd2.cuh", "swa_tile.cuh", "sm100.cuh"),
+    "fwd2_kernel": ("swa_fwd2.cuh", "sm100.cuh"),
     "decode_split_kernel": ("swa_decode.cuh", "sm100.cuh"),
 }
 

@@ -238,6 +238,15 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// 2^x for two values at once on the MUFU: x packed to bf16 (round to nearest),
+// result as packed bf16 -- the form the P operand of the PV MMA takes.
+__device__ __forceinline__ uint32_t ex2_bf16x2(float lo, float hi) {
+  uint32_t x, y;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

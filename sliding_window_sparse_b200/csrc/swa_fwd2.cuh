@@ -50,6 +50,10 @@ constexpr float kLazyRescaleLog2 = 8.0f;
 #ifndef SWA_EMU_COLS
 #define SWA_EMU_COLS 0
 #endif
+// Exponentials of P as packed bf16 pairs on the MUFU (ex2.approx.ftz.bf16x2).
+#ifndef SWA_EX2_BF16X2
+#define SWA_EX2_BF16X2 0
+#endif
 constexpr int kEmuCols = SWA_EMU_COLS;
 static_assert(kEmuCols % 16 == 0 && kEmuCols <= 128, "emulated columns in groups of 16");
 
@@ -414,10 +418,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         int k, src, y0, ca, cb, na = 0, nb = 0;
         bool have = wk.next_live(k, src, y0, ca, cb);
         bool first[2] = {true, true};
-        if (!have) {  // (no live tile: keep every barrier's phase count in step)
+        if (!have) {  // no live tile: keep the Q barriers' phase counts in step
           tc_commit(BAR_QE);
-          tc_commit(BAR_O);
-          tc_commit(BAR_O + 8);
           ++q_iter;
           continue;
         }
@@ -486,8 +488,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           have = has_next;
           if (have) has_next = wk.next_live(k, src, y0, na, nb);
         }
-        if (!o_done[0]) tc_commit(BAR_O);
-        if (!o_done[1]) tc_commit(BAR_O + 8);
+        // o_final completes once per unit in which the tile had work; its next
+        // completion needs that tile's softmax to hand over its next P, so it
+        // can never run two phases ahead of the waiting softmax warps
+        if (!first[0] && !o_done[0]) tc_commit(BAR_O);
+        if (!first[1] && !o_done[1]) tc_commit(BAR_O + 8);
         ++q_iter;
       }
     }
@@ -559,6 +564,33 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         float2 *s2 = reinterpret_cast<float2 *>(s);
 #pragma unroll
         for (int c = 0; c < kKT / 2; ++c) s2[c] = __ffma2_rn(s2[c], sc2, nm2);
+#if SWA_EX2_BF16X2
+        // P = 2^x evaluated two columns per MUFU op directly in bf16 (the PV MMA's
+        // operand type); the row sum adds exactly those bf16 weights
+        uint32_t pk[kKT / 2];
+#pragma unroll
+        for (int c = 0; c < kKT / 2; ++c) pk[c] = ex2_bf16x2(s2[c].x, s2[c].y);
+        float2 sm2[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kKT / 2; c += 4)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            sm2[i] = __fadd2_rn(sm2[i], make_float2(__uint_as_float(pk[c + i] << 16),
+                                                    __uint_as_float(pk[c + i] & 0xFFFF0000u)));
+        const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
+        const float rs = sa.x + sa.y;
+        l_run = l_run * alpha + rs;
+        m_run = m_new;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t half[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) half[i] = pk[h2 * 32 + i];
+          tmem_st32(tS + h2 * 32, half);
+        }
+#else
         // exponentials: MUFU for the first columns, FMA-pipe polynomial for the last
         // kEmuCols (a masked column clamps to 2^-125 there, which is numerically 0
         // next to the row maximum's 2^0 and is cleared with O and l by any later
@@ -587,6 +619,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[h2 * 64 + 2 * i], s[h2 * 64 + 2 * i + 1]);
           tmem_st32(tS + h2 * 32, pk);
         }
+#endif
         // O_X is stable: PV_X of the previous tile was issued before this S_X
         if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -604,11 +637,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         mbar_arrive(BAR_P + 8 * x);
         ++nt;
       }
-      // every PV of this unit is done
-      mbar_wait(BAR_O + 8 * x, u_iter & 1, abort_flag);
-      ++u_iter;
-      tc_fence_after();
       if (nt > 0) {
+        // every PV of this unit is done
+        mbar_wait(BAR_O + 8 * x, u_iter & 1, abort_flag);
+        ++u_iter;
+        tc_fence_after();
         const float inv_l = 1.f / l_run;
         const int hh = U.h[x];
         __nv_bfloat16 *orow =
