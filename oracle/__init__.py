@@ -22,6 +22,11 @@ Functions and the passages they follow (page title, section):
 * :func:`ring_update`     -- Chapter 10 section 10.2; blog section 3.2.
 * :func:`swa_decode`      -- blog section 3.2; taxonomy page section 1.
 * :func:`tile_classes`    -- M003 note section 04 (skip / full / partial tiles).
+* :func:`count_pairs_sink` -- taxonomy page section 3.2 (StreamingLLM: first
+                             tokens plus the recent W), by enumeration.
+* :func:`swa_varlen`      -- blog section 5.2 tip 4 (packed batches, windows per
+                             sequence via cu_seqlens), with optional sinks.
+* :func:`swa_decode_sink` -- taxonomy page section 3.2 on top of the ring decode.
 
 All of them are pinned by ``tests/test_oracle_pins.py``.
 """
@@ -90,6 +95,14 @@ def _configure(lib):
     lib.orc_swa_decode.restype = _i64
     lib.orc_swa_decode.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int, _i64,
                                    _dbl, _ptr, _ptr]
+    lib.orc_count_pairs_sink.restype = _i64
+    lib.orc_count_pairs_sink.argtypes = [_i64, _i64, _i64]
+    lib.orc_swa_varlen.restype = _i64
+    lib.orc_swa_varlen.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int, _i64, _i64,
+                                   _dbl, _ptr, _i64, _ptr, _ptr]
+    lib.orc_swa_decode_sink.restype = _i64
+    lib.orc_swa_decode_sink.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int,
+                                        _int, _i64, _i64, _dbl, _ptr, _ptr]
     lib.orc_tile_classes.restype = _int
     lib.orc_tile_classes.argtypes = [_int, _int, _i64, _i64, _ptr, _i64, _int, _int, _ptr,
                                      _ptr]
@@ -172,6 +185,42 @@ def swa_forward(q, k, v, W: int, scale: float, rows=None, q_pos0=None, with_lse=
     return (out, lse) if with_lse else out
 
 
+def count_pairs_sink(N: int, W: int, n_sink: int) -> int:
+    """Visible pairs among N positions with the window plus the first n_sink keys."""
+    return int(_load().orc_count_pairs_sink(N, W, n_sink))
+
+
+def swa_varlen(q, k, v, cu_seqlens, W: int, scale: float, n_sink: int = 0, rows=None,
+               with_lse=False):
+    """Packed variable-length attention, per-sequence windows (and sinks).
+
+    q: [total,H,d], k/v: [total,Hkv,d] bf16 bits; cu_seqlens: [n_seq+1] int64 from 0.
+    ``rows``: optional (n,2) int64 array of (token, h); the result is then [n, d]
+    instead of [total,H,d] (lse [n] instead of [total,H]).
+    """
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    total, H, d = q.shape
+    Hkv = k.shape[1]
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64).reshape(-1)
+    if cu[-1] != total:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    n = r.shape[0] if r is not None else total * H
+    out = np.empty((n, d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64) if with_lse else None
+    bad = _load().orc_swa_varlen(_p(q), _p(k), _p(v), _p(cu), cu.shape[0] - 1, H, Hkv, d, W,
+                                 n_sink, scale, _p(r), n, _p(out), _p(lse))
+    if bad < 0:
+        raise ValueError("cu_seqlens must start at 0 and be non-decreasing")
+    if bad:
+        raise ValueError(f"{bad} query rows have no legal key")
+    if r is None:
+        out = out.reshape(total, H, d)
+        if lse is not None:
+            lse = lse.reshape(total, H)
+    return (out, lse) if with_lse else out
+
+
 def dense_masked(q, k, v, W: int, scale: float):
     """Dense score table + window mask + row softmax (positions 0..N-1)."""
     q, k, v = _u16(q), _u16(k), _u16(v)
@@ -233,6 +282,23 @@ def swa_decode(q, ring_k, ring_v, pos, W: int, scale: float, with_lse=False):
     lse = np.empty((B, H), dtype=np.float64) if with_lse else None
     bad = _load().orc_swa_decode(_p(q), _p(ring_k), _p(ring_v), _p(p), B, H, Hkv, d, W, scale,
                                  _p(out), _p(lse))
+    if bad:
+        raise ValueError(f"{bad} decode rows have a missing or no legal key")
+    return (out, lse) if with_lse else out
+
+
+def swa_decode_sink(q, ring_k, ring_v, sink_k, sink_v, pos, W: int, scale: float,
+                    with_lse=False):
+    """Decode over a ring plus sink rows [B,Hkv,S,d] holding positions 0..S-1."""
+    q, ring_k, ring_v = _u16(q), _u16(ring_k), _u16(ring_v)
+    sink_k, sink_v = _u16(sink_k), _u16(sink_v)
+    B, H, d = q.shape
+    Hkv, S = sink_k.shape[1], sink_k.shape[2]
+    p = np.ascontiguousarray(pos, dtype=np.int64).reshape(B)
+    out = np.empty((B, H, d), dtype=np.float64)
+    lse = np.empty((B, H), dtype=np.float64) if with_lse else None
+    bad = _load().orc_swa_decode_sink(_p(q), _p(ring_k), _p(ring_v), _p(sink_k), _p(sink_v),
+                                      _p(p), B, H, Hkv, d, W, S, scale, _p(out), _p(lse))
     if bad:
         raise ValueError(f"{bad} decode rows have a missing or no legal key")
     return (out, lse) if with_lse else out

@@ -17,7 +17,11 @@
  *  [CH10]  "Chapter 10 -- local and sparse attention: SWA and DSA"
  *          (book.ozine.me, LLMs from scratch), sections 10.1, 10.2, 10.3, 10.6.
  *  [BLOG]  "Dense attention vs sparse sliding window attention"
- *          (maplevalley.com.cn news 3171860), section 3.2 (circular KV cache).
+ *          (maplevalley.com.cn news 3171860), section 3.2 (circular KV cache),
+ *          section 5.2 tip 4 (per-sequence windows in packed batches).
+ *  [TAXO]  "Sparse attention taxonomy: what to read, what not to read"
+ *          (forceinjection.github.io, kv_cache concepts), section 3.2
+ *          (StreamingLLM: the first 4 tokens plus the recent W).
  *
  * Parity pins for every function live in tests/test_oracle_pins.py.
  */
@@ -368,6 +372,139 @@ int64_t orc_swa_decode(const uint16_t *q, const uint16_t *ring_k, const uint16_t
                 if (s < 0) { ++missing; continue; }
                 kr[n] = ring_k + ((b * Hkv + kh) * W + s) * d;
                 vr[n] = ring_v + ((b * Hkv + kh) * W + s) * d;
+                ++n;
+            }
+            int e = attend_one(q + (b * H + h) * d, kr, vr, n, d, scale, out + r * d,
+                               lse ? lse + r : NULL, sc);
+            if (e || missing) ++bad;
+        }
+        free(kr);
+        free(vr);
+        free(sc);
+    }
+    free(maps);
+    return bad;
+}
+
+/* [M003 s03] with StreamingLLM's sink rule ([TAXO s3.2], StreamingLLM:
+ * the first S tokens stay visible besides the recent W): key j is visible to
+ * position i iff j <= i and (j >= i - W + 1 or j < S).  S = 0 is allowed(). */
+static int allowed_sink(int64_t i, int64_t j, int64_t W, int64_t S)
+{
+    return (j <= i) && (j >= 0) && (j >= i - W + 1 || j < S);
+}
+
+/* Pairs visible under allowed_sink among all N x N positions, by enumeration. */
+int64_t orc_count_pairs_sink(int64_t N, int64_t W, int64_t S)
+{
+    int64_t n = 0;
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t j = 0; j < N; ++j)
+            n += allowed_sink(i, j, W, S);
+    return n;
+}
+
+/*
+ * Packed variable-length prefill ([BLOG s5.2] tip 4: batches of
+ * different lengths packed along one token axis with cu_seqlens; the window
+ * is applied within each sequence, never across a boundary).
+ * q: [total, H, d]; k, v: [total, Hkv, d] (bf16 bits, token-major).
+ * Sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1] - 1, at positions
+ * 0, 1, ...  Query token t of sequence s (position i = t - cu_seqlens[s])
+ * reads the tokens cu_seqlens[s] + j with allowed_sink(i, j, W, n_sink), in
+ * increasing j.
+ * rows: pairs (t, h), or NULL for every (t, h) with h fastest.
+ * out: [n_rows, d] (or [total, H, d]); lse: [n_rows] (or [total, H]), optional.
+ * Returns the number of rows with no legal key, or -1 if cu_seqlens is not
+ * non-decreasing from 0.
+ */
+int64_t orc_swa_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int64_t *cu_seqlens, int n_seq, int H, int Hkv, int d, int64_t W,
+                       int64_t n_sink, double scale, const int64_t *rows, int64_t n_rows,
+                       double *out, double *lse)
+{
+    if (cu_seqlens[0] != 0) return -1;
+    int64_t longest = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (len < 0) return -1;
+        if (len > longest) longest = len;
+    }
+    int64_t total_tok = cu_seqlens[n_seq];
+    int64_t total = rows ? n_rows : total_tok * H;
+    int64_t bad = 0;
+#pragma omp parallel reduction(+ : bad)
+    {
+        int64_t cap = longest > 0 ? longest : 1;
+        const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)cap);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < total; ++r) {
+            int64_t t = rows ? rows[2 * r] : r / H;
+            int64_t h = rows ? rows[2 * r + 1] : r % H;
+            int s = 0;
+            while (s + 1 < n_seq && cu_seqlens[s + 1] <= t) ++s;
+            int64_t first = cu_seqlens[s], len = cu_seqlens[s + 1] - first;
+            int64_t i = t - first, kh = kv_head(h, H, Hkv);
+            int64_t n = 0;
+            for (int64_t j = 0; j < len; ++j) {
+                if (!allowed_sink(i, j, W, n_sink)) continue;
+                kr[n] = k + ((first + j) * Hkv + kh) * d;
+                vr[n] = v + ((first + j) * Hkv + kh) * d;
+                ++n;
+            }
+            const uint16_t *qrow = q + (t * H + h) * d;
+            if (attend_one(qrow, kr, vr, n, d, scale, out + r * d, lse ? lse + r : NULL, sc))
+                ++bad;
+        }
+        free(kr);
+        free(vr);
+        free(sc);
+    }
+    return bad;
+}
+
+/*
+ * Decode with attention sinks ([TAXO s3.2]).  The ring holds the recent
+ * positions exactly as in orc_swa_decode; sink_k, sink_v: [B, Hkv, S, d] hold
+ * positions 0 .. S-1, written once and never overwritten.  The query at
+ * pos[b] reads every position j with allowed_sink(pos[b], j, W, S) in
+ * increasing order: from the ring if j is one of the last W positions, else
+ * (a sink outside the window) from the sink rows.
+ * q: [B,H,d]; out: [B,H,d]; lse: [B,H] optional.
+ */
+int64_t orc_swa_decode_sink(const uint16_t *q, const uint16_t *ring_k, const uint16_t *ring_v,
+                            const uint16_t *sink_k, const uint16_t *sink_v, const int64_t *pos,
+                            int B, int H, int Hkv, int d, int64_t W, int64_t S, double scale,
+                            double *out, double *lse)
+{
+    int64_t bad = 0;
+    int64_t *maps = (int64_t *)malloc(sizeof(int64_t) * (size_t)(B * W));
+    for (int64_t b = 0; b < B; ++b) orc_ring_positions(pos[b] + 1, W, maps + b * W);
+#pragma omp parallel reduction(+ : bad)
+    {
+        int64_t cap = W + S;
+        const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)cap);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < (int64_t)B * H; ++r) {
+            int64_t b = r / H, h = r % H;
+            int64_t kh = kv_head(h, H, Hkv);
+            int64_t p = pos[b];
+            int64_t n = 0, missing = 0;
+            for (int64_t j = 0; j <= p; ++j) {
+                if (!allowed_sink(p, j, W, S)) continue;
+                if (j >= p - W + 1) {
+                    int64_t s = find_slot(maps + b * W, W, j);
+                    if (s < 0) { ++missing; continue; }
+                    kr[n] = ring_k + ((b * Hkv + kh) * W + s) * d;
+                    vr[n] = ring_v + ((b * Hkv + kh) * W + s) * d;
+                } else {
+                    kr[n] = sink_k + ((b * Hkv + kh) * S + j) * d;
+                    vr[n] = sink_v + ((b * Hkv + kh) * S + j) * d;
+                }
                 ++n;
             }
             int e = attend_one(q + (b * H + h) * d, kr, vr, n, d, scale, out + r * d,

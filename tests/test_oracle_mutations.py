@@ -43,6 +43,16 @@ MUTANTS = {
         "int64_t r_end = r_begin + tile_q < n_q ? r_begin + tile_q : n_q;",
         "int64_t r_end = r_begin + tile_q - 1 < n_q ? r_begin + tile_q - 1 : n_q;"),
     "count_pairs_strict": ("n += allowed(i, j, W);", "n += allowed(i, j, W) && j < i;"),
+    "sink_count_inclusive": ("(j >= i - W + 1 || j < S)", "(j >= i - W + 1 || j <= S)"),
+    "sink_pairs_ignore_sinks": ("n += allowed_sink(i, j, W, S);", "n += allowed(i, j, W);"),
+    "varlen_sequence_base_dropped": ("kr[n] = k + ((first + j) * Hkv + kh) * d;",
+                                     "kr[n] = k + (j * Hkv + kh) * d;"),
+    "varlen_boundary_token_misassigned": (
+        "while (s + 1 < n_seq && cu_seqlens[s + 1] <= t) ++s;",
+        "while (s + 1 < n_seq && cu_seqlens[s + 1] < t) ++s;"),
+    "decode_sink_row_fixed": ("kr[n] = sink_k + ((b * Hkv + kh) * S + j) * d;",
+                              "kr[n] = sink_k + ((b * Hkv + kh) * S + 0) * d;"),
+    "decode_sink_window_edge": ("if (j >= p - W + 1) {", "if (j > p - W + 1) {"),
 }
 
 
@@ -67,6 +77,16 @@ def _pin_suite(golden_dir):
         lambda: pins.test_full_equals_chunked_general(16, [(0, 5), (5, 40), (40, 41), (41, 90)]),
         lambda: pins.test_decode_equals_prefill_row(16, 50),
         lambda: pins.test_lse_matches_definition(),
+        lambda: pins.test_sink_pairs_closed_form(100, 7, 4),
+        lambda: pins.test_sink_pairs_special_cases(),
+        lambda: pins.test_varlen_visible_sets([8, 5, 1, 12], 3, 4),
+        lambda: pins.test_varlen_first_token_returns_own_value(),
+        lambda: pins.test_varlen_single_sequence_equals_linear_forward(),
+        lambda: pins.test_varlen_reduces_to_causal_sdpa(1000, 0),
+        lambda: pins.test_varlen_no_cross_talk(),
+        lambda: pins.test_sink_tokens_influence_and_middle_tokens_do_not(),
+        lambda: pins.test_decode_sink_equals_prefill_row(8, 4, 12),
+        lambda: pins.test_decode_sink_equals_prefill_row(16, 4, 50),
     ]
 
 

@@ -379,6 +379,176 @@ def test_lse_matches_definition():
             assert abs(lse[0, h, i] - math.log(sum(math.exp(x) for x in s))) < 1e-12
 
 
+# --- sinks (taxonomy page section 3.2: first tokens + recent W) ---------------
+
+def _sink_pairs_closed_form(N, W, S):
+    """Window pairs N*W - W(W-1)/2 (N >= W) plus, for query i >= W, the
+    min(S, i - W + 1) sink keys that lie before its window."""
+    if W >= N:
+        return N * (N + 1) // 2
+    m = N - W  # queries whose window does not reach position 0
+    extra = m * (m + 1) // 2 if m <= S else S * (S + 1) // 2 + (m - S) * S
+    return N * W - W * (W - 1) // 2 + extra
+
+
+@pytest.mark.parametrize("N,W,S", [(8, 3, 1), (8, 3, 4), (8, 3, 0), (100, 7, 4), (64, 64, 4),
+                                   (50, 1, 4), (30, 5, 30), (1000, 16, 4)])
+def test_sink_pairs_closed_form(N, W, S):
+    assert oracle.count_pairs_sink(N, W, S) == _sink_pairs_closed_form(N, W, S)
+
+
+def test_sink_pairs_special_cases():
+    # no sinks: the plain window; sinks covering everything: full causal
+    for N, W in [(8, 3), (100, 7), (33, 1)]:
+        assert oracle.count_pairs_sink(N, W, 0) == oracle.count_pairs(N, W)
+        assert oracle.count_pairs_sink(N, W, N) == N * (N + 1) // 2
+    # N = 8, W = 3, one sink: queries 3..7 each gain key 0 (21 + 5)
+    assert oracle.count_pairs_sink(8, 3, 1) == 26
+
+
+def _varlen_support(lens, W, S):
+    """Visible token sets per query token, read off the oracle with zero scores
+    and one-hot values (as _support_sets, over a packed batch)."""
+    total = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q = _bits(np.zeros((total, 1, total)))
+    k = _bits(np.zeros((total, 1, total)))
+    v = _bits(np.eye(total).reshape(total, 1, total))
+    out = oracle.swa_varlen(q, k, v, cu, W, 1.0, n_sink=S)
+    sets = []
+    for t in range(total):
+        row = out[t, 0]
+        support = [int(j) for j in np.nonzero(row > 0)[0]]
+        assert np.allclose(row[support], 1.0 / len(support), atol=1e-15)
+        sets.append(support)
+    return cu, sets
+
+
+@pytest.mark.parametrize("lens,W,S", [([8], 3, 1), ([8, 5, 1, 12], 3, 4), ([20, 20], 6, 2),
+                                      ([3, 0, 9], 2, 0)])
+def test_varlen_visible_sets(lens, W, S):
+    """Token t of sequence s sees, inside s only, the first S positions and the
+    recent W (the current one included) -- never a token of another sequence."""
+    cu, sets = _varlen_support(lens, W, S)
+    for s in range(len(lens)):
+        for i in range(lens[s]):
+            want = sorted({j for j in range(i + 1) if j < S or j >= i - W + 1})
+            assert sets[cu[s] + i] == [int(cu[s]) + j for j in want]
+
+
+def test_varlen_first_token_returns_own_value():
+    """The first token of every sequence has one legal key: itself."""
+    lens = [5, 1, 17, 9]
+    total = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q = _rand(21, (total, 4, 16), si.STREAM["q"])
+    k = _rand(21, (total, 2, 16), si.STREAM["k"])
+    v = _rand(21, (total, 2, 16), si.STREAM["v"])
+    out = oracle.swa_varlen(q, k, v, cu, 4, 0.25, n_sink=2)
+    vf = si.bf16_bits_to_f32(v).astype(np.float64)
+    for s in range(len(lens)):
+        t = int(cu[s])
+        for h in range(4):
+            assert np.array_equal(out[t, h], vf[t, h // 2])
+
+
+def test_varlen_single_sequence_equals_linear_forward():
+    """One sequence, no sinks: the [total,H,d] result is the [1,H,N,d] one."""
+    N, H, Hkv, d, W = 70, 4, 2, 16, 9
+    q = _rand(22, (1, H, N, d), si.STREAM["q"])
+    k = _rand(22, (1, Hkv, N, d), si.STREAM["k"])
+    v = _rand(22, (1, Hkv, N, d), si.STREAM["v"])
+    ref = oracle.swa_forward(q, k, v, W, 0.3)
+    tm = lambda x: np.ascontiguousarray(x[0].transpose(1, 0, 2))
+    got = oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, 0.3)
+    assert np.array_equal(got, ref[0].transpose(1, 0, 2))
+
+
+@pytest.mark.parametrize("W,S", [(1000, 0), (3, 1000)])
+def test_varlen_reduces_to_causal_sdpa(W, S):
+    """A window or a sink count covering every sequence is causal attention,
+    sequence by sequence (torch scaled-dot-product attention in fp64)."""
+    import torch
+
+    lens = [37, 1, 64, 20]
+    H, Hkv, d = 4, 2, 16
+    total = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q = _rand(23, (total, H, d), si.STREAM["q"])
+    k = _rand(23, (total, Hkv, d), si.STREAM["k"])
+    v = _rand(23, (total, Hkv, d), si.STREAM["v"])
+    scale = 0.25
+    got = oracle.swa_varlen(q, k, v, cu, W, scale, n_sink=S)
+    for s, n in enumerate(lens):
+        a, b = int(cu[s]), int(cu[s + 1])
+        tq, tk, tv = (torch.from_numpy(si.bf16_bits_to_f32(x[a:b]).astype(np.float64))
+                      .permute(1, 0, 2).unsqueeze(0) for x in (q, k, v))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk, tv, is_causal=True, scale=scale, enable_gqa=True)[0].permute(1, 0, 2).numpy()
+        assert np.max(np.abs(got[a:b] - ref)) < 1e-12
+
+
+def test_varlen_no_cross_talk():
+    """Changing one sequence's tokens leaves every other sequence's output as it was."""
+    lens = [30, 12, 25]
+    total = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q = _rand(24, (total, 2, 8), si.STREAM["q"])
+    k = _rand(24, (total, 2, 8), si.STREAM["k"])
+    v = _rand(24, (total, 2, 8), si.STREAM["v"])
+    base = oracle.swa_varlen(q, k, v, cu, 8, 0.5, n_sink=4)
+    k2, v2 = k.copy(), v.copy()
+    k2[30:42] = _rand(25, (12, 2, 8), si.STREAM["k"])
+    v2[30:42] = _rand(25, (12, 2, 8), si.STREAM["v"])
+    moved = oracle.swa_varlen(q, k2, v2, cu, 8, 0.5, n_sink=4)
+    assert np.array_equal(moved[:30], base[:30]) and np.array_equal(moved[42:], base[42:])
+    assert not np.array_equal(moved[30:42], base[30:42])
+
+
+def test_sink_tokens_influence_and_middle_tokens_do_not():
+    """Query i >= W + S: perturbing a sink changes it, perturbing a key strictly
+    between the sinks and the window does not."""
+    N, W, S = 40, 8, 4
+    q = _rand(26, (N, 1, 8), si.STREAM["q"])
+    k = _rand(26, (N, 1, 8), si.STREAM["k"])
+    v = _rand(26, (N, 1, 8), si.STREAM["v"])
+    base = oracle.swa_varlen(q, k, v, [0, N], W, 0.5, n_sink=S)
+    for j, changes in [(0, True), (S - 1, True), (S, False), (N - 1 - W, False)]:
+        v2 = v.copy()
+        v2[j] = _rand(27 + j, (1, 1, 8), si.STREAM["v"])
+        got = oracle.swa_varlen(q, k, v2, [0, N], W, 0.5, n_sink=S)
+        assert (not np.array_equal(got[N - 1], base[N - 1])) == changes, j
+
+
+@pytest.mark.parametrize("W,S,P", [(16, 4, 50), (16, 4, 5), (8, 4, 11), (8, 4, 12), (1, 4, 9),
+                                   (16, 0, 30)])
+def test_decode_sink_equals_prefill_row(W, S, P):
+    """Decode over ring + sink rows equals the last row of the packed prefill
+    with the same sinks (and, for S = 0, the plain ring decode)."""
+    B, H, Hkv, d = 2, 4, 2, 8
+    N = P + 1
+    q = _rand(28, (B, H, N, d), si.STREAM["q"])
+    k = _rand(28, (B, Hkv, N, d), si.STREAM["k"])
+    v = _rand(28, (B, Hkv, N, d), si.STREAM["v"])
+    rk = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rv = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rk, rv = oracle.ring_update(k, v, rk, rv, [0] * B, W)
+    sk = np.zeros((B, Hkv, max(S, 1), d), dtype=np.uint16)[:, :, :S]
+    sv = sk.copy()
+    n_s = min(S, N)
+    sk[:, :, :n_s] = k[:, :, :n_s]
+    sv[:, :, :n_s] = v[:, :, :n_s]
+    dec = oracle.swa_decode_sink(np.ascontiguousarray(q[:, :, P]), rk, rv, sk, sv, [P] * B, W,
+                                 0.4)
+    for b in range(B):
+        tm = lambda x: np.ascontiguousarray(x[b].transpose(1, 0, 2))
+        full = oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, 0.4, n_sink=S)
+        assert np.array_equal(dec[b], full[P])
+    if S == 0:
+        plain = oracle.swa_decode(np.ascontiguousarray(q[:, :, P]), rk, rv, [P] * B, W, 0.4)
+        assert np.array_equal(dec, plain)
+
+
 # --- the generator itself ------------------------------------------------------
 
 def test_generator_reproducible_and_normal():
