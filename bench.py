@@ -10,7 +10,9 @@ TFLOP/s = 4 * d * valid_pairs * H * B / time, summed over ranks (each rank runs
 its own independent batch: weak scaling, no data-path collective).
 
 The same run also times the chunked-prefill-on-ring and decode paths (and the
-narrow-window prefill) on their workloads under "paths", prints one JSON line
+narrow-window prefill), then the packed variable-length prefill, prefill and
+decode with attention sinks and ragged chunks, each on its own workload, under
+"paths".  It prints one JSON line
 on rank 0, and adds the roofline fraction of the timed kernel, a CPU baseline
 (the fp64 oracle on a bounded sample of rows, timed on the host cores), an
 end-to-end figure through the public API with host buffers, and SM clocks
@@ -54,23 +56,49 @@ def valid_pairs_row(pos: int, W: int) -> int:
     return min(W, pos + 1)
 
 
-def valid_pairs(w) -> int:
-    """Allowed (query, key) pairs per (b, h): N*W - W*(W-1)/2 for N >= W."""
-    if w.kind == "prefill":
-        N, W = w.N, w.W
-        return N * W - W * (W - 1) // 2 if N >= W else N * (N + 1) // 2
-    if w.kind == "chunk":
-        return sum(valid_pairs_row(p, w.W) for p in range(w.q_start, w.q_start + w.Tq))
-    return w.W
+def sequence_pairs(N: int, W: int, S: int = 0) -> int:
+    """Visible (query, key) pairs of one sequence of N positions: N*W - W*(W-1)/2
+    window pairs (N >= W), plus min(S, i - W + 1) sinks before the window of
+    each query i >= W."""
+    base = N * W - W * (W - 1) // 2 if N >= W else N * (N + 1) // 2
+    m = max(0, N - W)
+    return base + (m * (m + 1) // 2 if m <= S else S * (S + 1) // 2 + (m - S) * S)
+
+
+def chunk_rows(w):
+    """Valid chunk rows per sequence."""
+    from swa_inputs.workloads import seq_lens
+
+    return [int(n) for n in seq_lens(w)] if w.len_hi else [w.Tq] * w.B
 
 
 def useful_flops(w) -> int:
-    return 4 * w.d * valid_pairs(w) * w.H * w.B
+    """4 * d * (visible pairs) * H, summed over the batch."""
+    if w.kind == "prefill":
+        return 4 * w.d * w.H * w.B * sequence_pairs(w.N, w.W, w.n_sink)
+    if w.kind == "varlen":
+        from swa_inputs.workloads import seq_lens
+
+        return 4 * w.d * w.H * sum(sequence_pairs(int(n), w.W, w.n_sink) for n in seq_lens(w))
+    if w.kind == "chunk":
+        pairs = sum(valid_pairs_row(w.q_start + t, w.W) for n in chunk_rows(w) for t in range(n))
+        return 4 * w.d * w.H * pairs
+    raise ValueError(w.kind)
+
+
+def decode_positions(w):
+    from swa_inputs import STREAM, uniform_int
+
+    return uniform_int(w.seed, STREAM["ctx_len"], w.B, w.ctx_lo, w.ctx_hi) - 1
 
 
 def decode_kv_bytes(w) -> int:
-    """K and V of every (b, kv head) read once: 2 tensors * B * Hkv * W * d * 2 bytes."""
-    return 2 * w.B * w.Hkv * w.W * w.d * 2
+    """K and V of every (b, kv head) read once: 2 tensors * B * Hkv * W * d * 2 bytes,
+    plus the sink rows that lie before each window."""
+    sinks = 0
+    if w.n_sink:
+        sinks = sum(min(w.n_sink, max(0, int(p) - w.W + 1)) for p in decode_positions(w))
+    return 2 * w.Hkv * w.d * 2 * (w.B * w.W + sinks)
 
 
 def algorithmic_bytes(w) -> int:
@@ -78,20 +106,32 @@ def algorithmic_bytes(w) -> int:
     e = 2
     if w.kind == "prefill":
         return e * w.d * w.B * (2 * w.H * w.N + 2 * w.Hkv * w.N)
+    if w.kind == "varlen":
+        from swa_inputs.workloads import cu_seqlens
+
+        total = int(cu_seqlens(w)[-1])
+        return e * w.d * (2 * w.H * total + 2 * w.Hkv * total)
     if w.kind == "chunk":
-        return e * w.d * w.B * (2 * w.H * w.Tq + 2 * w.Hkv * (w.Tq + w.W))
+        rows = sum(chunk_rows(w))
+        return e * w.d * (2 * w.H * rows + 2 * w.Hkv * (rows + w.B * w.W))
     return decode_kv_bytes(w) + e * w.d * w.B * w.H * 2
 
 
 # ----------------------------------------------------------------------------- helpers
 
 def describe(w) -> str:
+    sink = f" sinks{w.n_sink}" if w.n_sink else ""
     if w.kind == "prefill":
-        return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} N{w.N} d{w.d} W{w.W}"
+        return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} N{w.N} d{w.d} W{w.W}{sink}"
+    if w.kind == "varlen":
+        return (f"{w.name}: {w.n_seq} packed sequences, lengths U[{w.len_lo},{w.len_hi}], "
+                f"H{w.H} Hkv{w.Hkv} d{w.d} W{w.W}{sink}")
     if w.kind == "chunk":
+        rows = f" valid rows U[{w.len_lo},{w.len_hi}]" if w.len_hi else ""
         return (f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} Tq{w.Tq} d{w.d} W{w.W} "
-                f"q_start{w.q_start}")
-    return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} d{w.d} W{w.W} ctx U[{w.ctx_lo},{w.ctx_hi}]"
+                f"q_start{w.q_start}{rows}")
+    return (f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} d{w.d} W{w.W} "
+            f"ctx U[{w.ctx_lo},{w.ctx_hi}]{sink}")
 
 
 def load_peaks():
@@ -203,19 +243,34 @@ def make_inputs(w, device, seed_offset=0):
     if w.kind == "prefill":
         return {"q": g("q", (w.B, w.H, w.N, w.d)), "k": g("k", (w.B, w.Hkv, w.N, w.d)),
                 "v": g("v", (w.B, w.Hkv, w.N, w.d))}
+    if w.kind == "varlen":
+        from swa_inputs.workloads import cu_seqlens
+
+        cu = cu_seqlens(w)
+        total = int(cu[-1])
+        return {"q": g("q", (total, w.H, w.d)), "k": g("k", (total, w.Hkv, w.d)),
+                "v": g("v", (total, w.Hkv, w.d)),
+                "cu_seqlens": torch.tensor(cu, dtype=torch.int64, device=device)}
     if w.kind == "chunk":
-        return {"q": g("q", (w.B, w.H, w.Tq, w.d)),
-                "k_new": g("k_new", (w.B, w.Hkv, w.Tq, w.d)),
-                "v_new": g("v_new", (w.B, w.Hkv, w.Tq, w.d)),
-                "k_ring": g("k_ring", (w.B, w.Hkv, w.W, w.d)),
-                "v_ring": g("v_ring", (w.B, w.Hkv, w.W, w.d)),
-                "q_start": torch.full((w.B,), w.q_start, dtype=torch.int64, device=device)}
+        x = {"q": g("q", (w.B, w.H, w.Tq, w.d)),
+             "k_new": g("k_new", (w.B, w.Hkv, w.Tq, w.d)),
+             "v_new": g("v_new", (w.B, w.Hkv, w.Tq, w.d)),
+             "k_ring": g("k_ring", (w.B, w.Hkv, w.W, w.d)),
+             "v_ring": g("v_ring", (w.B, w.Hkv, w.W, w.d)),
+             "q_start": torch.full((w.B,), w.q_start, dtype=torch.int64, device=device)}
+        if w.len_hi:
+            x["chunk_len"] = torch.tensor(chunk_rows(w), dtype=torch.int64, device=device)
+        return x
     from swa_inputs import uniform_int
 
     ctx = uniform_int(s, STREAM["ctx_len"], w.B, w.ctx_lo, w.ctx_hi)
-    return {"q": g("q", (w.B, w.H, w.d)), "k_ring": g("k_ring", (w.B, w.Hkv, w.W, w.d)),
-            "v_ring": g("v_ring", (w.B, w.Hkv, w.W, w.d)),
-            "pos": torch.tensor(ctx - 1, dtype=torch.int64, device=device)}
+    x = {"q": g("q", (w.B, w.H, w.d)), "k_ring": g("k_ring", (w.B, w.Hkv, w.W, w.d)),
+         "v_ring": g("v_ring", (w.B, w.Hkv, w.W, w.d)),
+         "pos": torch.tensor(ctx - 1, dtype=torch.int64, device=device)}
+    if w.n_sink:
+        x["k_sink"] = g("k_sink", (w.B, w.Hkv, w.n_sink, w.d))
+        x["v_sink"] = g("v_sink", (w.B, w.Hkv, w.n_sink, w.d))
+    return x
 
 
 def make_call(w, x, swa):
@@ -224,9 +279,21 @@ def make_call(w, x, swa):
 
     if w.kind == "prefill":
         out = torch.empty_like(x["q"])
-        return lambda: swa.swa_attn_fwd(x["q"], x["k"], x["v"], w.W, w.scale, out=out), out, 1
+        return (lambda: swa.swa_attn_fwd(x["q"], x["k"], x["v"], w.W, w.scale, out=out,
+                                         n_sink=w.n_sink), out, 1)
+    if w.kind == "varlen":
+        from swa_inputs.workloads import seq_lens
+
+        out = torch.empty_like(x["q"])
+        max_len = int(max(seq_lens(w)))
+        return (lambda: swa.swa_attn_varlen(x["q"], x["k"], x["v"], x["cu_seqlens"], max_len,
+                                            w.W, w.scale, n_sink=w.n_sink, out=out), out, 1)
     if w.kind == "chunk":
         out = torch.empty_like(x["q"])
+        if "chunk_len" in x:
+            return (lambda: swa.swa_attn_chunk_ring_ragged(
+                x["q"], x["k_new"], x["v_new"], x["k_ring"], x["v_ring"], x["q_start"],
+                x["chunk_len"], w.scale, out=out), out, 1)
         return (lambda: swa.swa_attn_chunk_ring(x["q"], x["k_new"], x["v_new"], x["k_ring"],
                                                 x["v_ring"], x["q_start"], w.scale, out=out),
                 out, 1)
@@ -234,7 +301,8 @@ def make_call(w, x, swa):
     ws = torch.empty(swa.swa_decode_workspace_bytes(w.B, w.H, w.Hkv, w.d, w.W), dtype=torch.uint8,
                      device=x["q"].device)
     return (lambda: swa.swa_attn_decode_ring(x["q"], x["k_ring"], x["v_ring"], x["pos"], w.scale,
-                                             workspace=ws, out=out), out, 2)
+                                             workspace=ws, out=out, k_sink=x.get("k_sink"),
+                                             v_sink=x.get("v_sink")), out, 2)
 
 
 def time_steps(call, steps, warmup, flush, barrier):
@@ -268,7 +336,7 @@ def time_e2e(w, x, swa, steps, warmup):
     import torch
 
     dev = x["q"].device
-    names = [n for n in x if n != "pos" and n != "q_start"]
+    names = [n for n in x if x[n].dtype != torch.int64]  # positions and offsets stay put
     host = {n: x[n].cpu().pin_memory() for n in names}
     xs = dict(x)
     call, out, _ = make_call(w, xs, swa)
@@ -436,7 +504,9 @@ def run_native(args):
     # the other paths of the hot path, on their own workloads
     paths = {}
     if not args.headline_only:
-        for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring"):
+        for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring",
+                     "varlen_prefill", "mistral_prefill_sink", "chunk_ring_ragged",
+                     "decode_ring_sink"):
             if name == headline:
                 continue
             pw = WORKLOADS[name]
@@ -468,7 +538,7 @@ def run_native(args):
 
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline and w.kind == "prefill":
+        if world == 1 and not args.no_cpu_baseline and w.kind == "prefill" and not w.n_sink:
             import oracle
 
             host = host_prefill_inputs(x)

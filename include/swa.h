@@ -106,6 +106,46 @@ SWA_API int swa_attn_fwd(const void *q, const void *k, const void *v, void *out,
                  int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream);
 
 /*
+ * swa_attn_fwd_sink -- swa_attn_fwd with attention sinks.
+ * Passage: sparse-attention taxonomy page section 3.2 (StreamingLLM keeps the
+ * first tokens visible besides the recent W).  Query i reads key j iff
+ * j <= i and (j >= i - W + 1 or j < n_sink).
+ *   n_sink: 0 <= n_sink <= 128 (0 is swa_attn_fwd).
+ * Other arguments, layouts and limits as swa_attn_fwd.
+ */
+SWA_API int swa_attn_fwd_sink(const void *q, const void *k, const void *v, void *out, float *lse,
+                              int B, int H, int Hkv, int64_t N, int d, int64_t W, int n_sink,
+                              float scale, void *stream);
+
+/*
+ * swa_attn_varlen -- prefill over a packed batch of sequences of different
+ * lengths, each with its own window.
+ * Passage: "Dense attention vs sparse SWA" blog section 5.2, tip 4 (in a
+ * packed batch the window is per sequence; cu_seqlens must split the samples
+ * exactly or windows leak across them); M003 note section 03 within each
+ * sequence; sinks as swa_attn_fwd_sink.
+ *   q:   [total, H, d]   bf16, device (token-major)
+ *   k, v: [total, Hkv, d] bf16, device
+ *   cu_seqlens: int64 [n_seq + 1], device: sequence s is tokens
+ *        cu_seqlens[s] .. cu_seqlens[s+1] - 1, at positions 0, 1, ... of its
+ *        own; non-decreasing, cu_seqlens[n_seq] <= total, every length
+ *        <= max_seqlen (else SWA_ERR_DEVICE is set on the device and the
+ *        offending sequence is skipped).  Empty sequences are allowed.
+ *   out: [total, H, d] bf16, device; rows of tokens outside every sequence are
+ *        not written.
+ *   lse: [H, total] fp32, device, or NULL.
+ *   n_sink: 0 <= n_sink <= 128: the first n_sink positions of each sequence
+ *        stay visible to all of its later queries.
+ * Limits: 1 <= total < 2^31 - 256, 1 <= max_seqlen < 2^29.  Tokens of a
+ * neighbouring sequence share tiles with a sequence's edges and get weight
+ * zero, so all of q, k, v must be finite.
+ */
+SWA_API int swa_attn_varlen(const void *q, const void *k, const void *v,
+                            const int64_t *cu_seqlens, void *out, float *lse, int n_seq,
+                            int64_t total, int64_t max_seqlen, int H, int Hkv, int d, int64_t W,
+                            int n_sink, float scale, void *stream);
+
+/*
  * swa_attn_chunk_ring -- chunked prefill over a W-slot ring-buffer KV cache.
  * Passage: Chapter 10 section 10.2 (a chunk of T_q queries needs the union of
  * W + T_q - 1 keys; the persistent cache keeps only the last W); M003 note
@@ -124,12 +164,38 @@ SWA_API int swa_attn_fwd(const void *q, const void *k, const void *v, void *out,
  * the chunk rows whose positions are among the last W are written into slots
  * position mod W, so the ring then serves the next chunk or decode step.
  * The ring is only written when update_ring != 0.  Limits: 1 <= Tq < 2^29,
- * W < 2^29.
+ * W < 2^29.  Empty ring slots must hold finite values (a zero-filled cache
+ * does): a tile that mixes them with visible keys loads them and gives them
+ * weight zero, and 0 * inf is NaN.
  */
 SWA_API int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,
                         void *v_ring, const int64_t *q_start, void *out, float *lse, int B,
                         int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
                         int update_ring, void *stream);
+
+/*
+ * swa_attn_chunk_ring_ragged -- swa_attn_chunk_ring for a batch whose chunks
+ * have different lengths (Chapter 10 section 10.2 applied per sequence; the
+ * window is per sequence, as the blog's troubleshooting section 5.2 stresses
+ * for batched requests).
+ *   chunk_len: int64 [B], device: sequence b's chunk has chunk_len[b] valid
+ *              rows, 0 <= chunk_len[b] <= Tq (a value outside that range sets
+ *              SWA_ERR_DEVICE on the device).  Its queries t < chunk_len[b]
+ *              sit at q_start[b] + t and see the ring and the chunk keys
+ *              t' < chunk_len[b] only; rows t >= chunk_len[b] of q, k_new,
+ *              v_new are padding: they get weight zero (so, like empty ring
+ *              slots, they must be finite), their output rows and lse
+ *              entries are left unwritten, and update_ring writes only the
+ *              valid rows among the last W.  A sequence with chunk_len[b] = 0
+ *              costs no tile work.
+ * Other arguments, layouts and limits as swa_attn_chunk_ring; chunk_len may
+ * not be NULL.
+ */
+SWA_API int swa_attn_chunk_ring_ragged(const void *q, const void *k_new, const void *v_new,
+                                       void *k_ring, void *v_ring, const int64_t *q_start,
+                                       const int64_t *chunk_len, void *out, float *lse, int B,
+                                       int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                                       int update_ring, void *stream);
 
 /*
  * swa_ring_write -- append a chunk of keys/values to a ring cache.
@@ -144,8 +210,9 @@ SWA_API int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, v
                    void *stream);
 
 /*
- * swa_decode_workspace_bytes -- bytes of scratch swa_attn_decode_ring needs
- * for these sizes (split partial results: fp32 O, running max and sum).
+ * swa_decode_workspace_bytes -- bytes of scratch swa_attn_decode_ring and
+ * swa_attn_decode_ring_sink need for these sizes (split partial results:
+ * fp32 O, running max and sum; one spare partial per (b, h) for sinks).
  */
 SWA_API size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int64_t W);
 
@@ -168,6 +235,24 @@ SWA_API int swa_attn_decode_ring(const void *q, const void *k_ring, const void *
                          const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
                          int d, int64_t W, float scale, void *workspace,
                          size_t workspace_bytes, void *stream);
+
+/*
+ * swa_attn_decode_ring_sink -- swa_attn_decode_ring with attention sinks.
+ * Passage: sparse-attention taxonomy page section 3.2 (StreamingLLM keeps the
+ * first tokens visible besides the recent W).  The query at pos[b] reads key
+ * j iff j <= pos[b] and (j >= pos[b] - W + 1 or j < n_sink): the last W
+ * positions from the ring, the sinks before the window from k_sink/v_sink.
+ *   k_sink, v_sink: [B, Hkv, n_sink, d] bf16, device: row j holds position j
+ *      (written once by the caller, e.g. copied from the first chunk; rows
+ *      j > pos[b] are never read).   1 <= n_sink <= 128.
+ * Other arguments, layouts and limits as swa_attn_decode_ring; the same
+ * workspace size applies.  One extra CTA per (b, kv head) reads the sinks.
+ */
+SWA_API int swa_attn_decode_ring_sink(const void *q, const void *k_ring, const void *v_ring,
+                                      const void *k_sink, const void *v_sink, int n_sink,
+                                      const int64_t *pos, void *out, float *lse, int B, int H,
+                                      int Hkv, int d, int64_t W, float scale, void *workspace,
+                                      size_t workspace_bytes, void *stream);
 
 /*
  * swa_attn_decode_ring_static -- swa_attn_decode_ring without a workspace.

@@ -25,10 +25,14 @@ __all__ = [
     "lib",
     "swa_block_meta",
     "swa_attn_fwd",
+    "swa_attn_fwd_sink",
+    "swa_attn_varlen",
     "swa_attn_chunk_ring",
+    "swa_attn_chunk_ring_ragged",
     "swa_ring_write",
     "swa_decode_workspace_bytes",
     "swa_attn_decode_ring",
+    "swa_attn_decode_ring_sink",
     "swa_attn_decode_ring_static",
     "swa_ring_slot_positions",
     "swa_get_device_status",
@@ -87,8 +91,11 @@ def swa_block_meta(key_mode: int, n_q: int, n_k: int, W: int, tile_q: int, tile_
 
 
 def swa_attn_fwd(q, k, v, W: int, scale: float | None = None, out=None, lse=None,
-                 return_lse: bool = False):
-    """Prefill forward: q [B,H,N,d], k/v [B,Hkv,N,d] -> out [B,H,N,d] (and lse [B,H,N])."""
+                 return_lse: bool = False, n_sink: int = 0):
+    """Prefill forward: q [B,H,N,d], k/v [B,Hkv,N,d] -> out [B,H,N,d] (and lse [B,H,N]).
+
+    n_sink > 0 keeps keys 0..n_sink-1 visible to every later query (swa_attn_fwd_sink).
+    """
     _need(q, "q", dims=4)
     _need(k, "k", dims=4)
     _need(v, "v", dims=4)
@@ -105,8 +112,45 @@ def swa_attn_fwd(q, k, v, W: int, scale: float | None = None, out=None, lse=None
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32, 3)
-    check("swa_attn_fwd", lib().swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H,
-                                             Hkv, N, d, W, scale, _stream(q.device)))
+    if n_sink:
+        check("swa_attn_fwd_sink",
+              lib().swa_attn_fwd_sink(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv,
+                                      N, d, W, n_sink, scale, _stream(q.device)))
+    else:
+        check("swa_attn_fwd", lib().swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                                 B, H, Hkv, N, d, W, scale, _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_attn_varlen(q, k, v, cu_seqlens, max_seqlen: int, W: int, scale: float | None = None,
+                    n_sink: int = 0, out=None, lse=None, return_lse: bool = False):
+    """Packed prefill: q [total,H,d], k/v [total,Hkv,d], cu_seqlens int64 [n_seq+1] (device).
+
+    Each sequence has its own positions and window; returns out [total,H,d] (and
+    lse [H,total]).  Rows of tokens outside every sequence keep what `out` held.
+    """
+    _need(q, "q", dims=3)
+    _need(k, "k", dims=3)
+    _need(v, "v", dims=3)
+    _need(cu_seqlens, "cu_seqlens", torch.int64, 1)
+    total, H, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (total, Hkv, d) or tuple(v.shape) != (total, Hkv, d):
+        raise ValueError("k and v must be [total, Hkv, d] matching q")
+    n_seq = cu_seqlens.shape[0] - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.zeros_like(q)
+    _need(out, "out", dims=3)
+    if return_lse and lse is None:
+        lse = torch.zeros((H, total), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    check("swa_attn_varlen",
+          lib().swa_attn_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+                                n_seq, total, max_seqlen, H, Hkv, d, W, n_sink, scale,
+                                _stream(q.device)))
     return (out, lse) if return_lse else out
 
 
@@ -132,6 +176,35 @@ def swa_attn_chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, scale: float |
     return (out, lse) if return_lse else out
 
 
+def swa_attn_chunk_ring_ragged(q, k_new, v_new, k_ring, v_ring, q_start, chunk_len,
+                               scale: float | None = None, update_ring: bool = False, out=None,
+                               lse=None, return_lse: bool = False):
+    """swa_attn_chunk_ring with chunk_len [B] valid rows per sequence (the rest is padding).
+
+    Output rows at or beyond chunk_len[b] are left as they were in `out` (zeros when `out` is
+    allocated here), likewise their lse entries.
+    """
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"),
+                 (v_ring, "v_ring")):
+        _need(t, n, dims=4)
+    _need(q_start, "q_start", torch.int64, 1)
+    _need(chunk_len, "chunk_len", torch.int64, 1)
+    B, H, Tq, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.zeros_like(q)
+    if return_lse and lse is None:
+        lse = torch.zeros((B, H, Tq), dtype=torch.float32, device=q.device)
+    check("swa_attn_chunk_ring_ragged",
+          lib().swa_attn_chunk_ring_ragged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring),
+                                           _ptr(v_ring), _ptr(q_start), _ptr(chunk_len),
+                                           _ptr(out), _ptr(lse), B, H, Hkv, Tq, d, W, scale,
+                                           1 if update_ring else 0, _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
 def swa_ring_write(k_new, v_new, k_ring, v_ring, q_start):
     """Write the chunk rows among the last W positions into slot position mod W (in place)."""
     for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"), (v_ring, "v_ring")):
@@ -149,8 +222,13 @@ def swa_decode_workspace_bytes(B: int, H: int, Hkv: int, d: int, W: int) -> int:
 
 
 def swa_attn_decode_ring(q, k_ring, v_ring, pos, scale: float | None = None, workspace=None,
-                         out=None, lse=None, return_lse: bool = False):
-    """Decode: q [B,H,d] at positions pos [B] over ring caches [B,Hkv,W,d] -> out [B,H,d]."""
+                         out=None, lse=None, return_lse: bool = False, k_sink=None,
+                         v_sink=None):
+    """Decode: q [B,H,d] at positions pos [B] over ring caches [B,Hkv,W,d] -> out [B,H,d].
+
+    With k_sink / v_sink [B,Hkv,S,d] (positions 0..S-1) the sinks before the window are
+    attended too (swa_attn_decode_ring_sink).
+    """
     _need(q, "q", dims=3)
     _need(k_ring, "k_ring", dims=4)
     _need(v_ring, "v_ring", dims=4)
@@ -166,11 +244,20 @@ def swa_attn_decode_ring(q, k_ring, v_ring, pos, scale: float | None = None, wor
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
-    check("swa_attn_decode_ring",
-          lib().swa_attn_decode_ring(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(pos), _ptr(out),
-                                     _ptr(lse), B, H, Hkv, d, W, scale, _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(),
-                                     _stream(q.device)))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if k_sink is not None:
+        _need(k_sink, "k_sink", dims=4)
+        _need(v_sink, "v_sink", dims=4)
+        check("swa_attn_decode_ring_sink",
+              lib().swa_attn_decode_ring_sink(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(k_sink),
+                                              _ptr(v_sink), k_sink.shape[2], _ptr(pos), _ptr(out),
+                                              _ptr(lse), B, H, Hkv, d, W, scale, _ptr(workspace),
+                                              ws_bytes, _stream(q.device)))
+    else:
+        check("swa_attn_decode_ring",
+              lib().swa_attn_decode_ring(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(pos),
+                                         _ptr(out), _ptr(lse), B, H, Hkv, d, W, scale,
+                                         _ptr(workspace), ws_bytes, _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

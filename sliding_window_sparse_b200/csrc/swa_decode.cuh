@@ -6,7 +6,10 @@
 // all G query heads of the group from the same registers.  The slot range of
 // one (b, kv head) is cut into `splits` CTAs; each writes an unnormalised
 // partial (o, running max m, running sum l, base 2) to the workspace, and
-// decode_combine_kernel merges them.
+// decode_combine_kernel merges them.  With attention sinks (sparse-attention
+// taxonomy page, section 3.2: StreamingLLM keeps the first tokens besides the
+// recent W) one more CTA per (b, kv head) streams the sink rows that lie
+// before the window, as one more partial.
 //
 // Warp layout: a key row of D bf16 is read by LPK = D / 8 lanes (16 bytes
 // each), so one warp-wide load covers KPW = 32 / LPK consecutive slots.  Lane
@@ -32,15 +35,19 @@ struct DecodeParams {
   const __nv_bfloat16 *q;       // [B, H, D]
   const __nv_bfloat16 *k_ring;  // [B, Hkv, W, D]
   const __nv_bfloat16 *v_ring;  // [B, Hkv, W, D]
+  const __nv_bfloat16 *k_sink;  // [B, Hkv, n_sink, D] positions 0 .. n_sink-1, or nullptr
+  const __nv_bfloat16 *v_sink;
   const int64_t *pos;           // [B]
-  float *ws_o;                  // [B*H, splits, D]
-  float *ws_ml;                 // [B*H, splits, 2]  (m, l) base-2 domain
+  float *ws_o;                  // [B*H, n_part, D]
+  float *ws_ml;                 // [B*H, n_part, 2]  (m, l) base-2 domain
   __nv_bfloat16 *out;           // [B, H, D]
   float *lse;                   // [B, H] or nullptr
   int B, H, Hkv;
   int64_t W;
   int chunk;   // slots per split CTA
-  int splits;  // CTAs per (b, kv head)
+  int splits;  // ring CTAs per (b, kv head)
+  int n_sink;  // sink rows (0: none)
+  int n_part;  // partials per (b, h): splits, plus one for the sinks
   float scale_log2;
 };
 
@@ -96,9 +103,16 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const Deco
     nvalid = 0;
     if (threadIdx.x == 0 && split == 0 && kvh == 0) atomicOr(&g_swa_status, SWA_DEV_BADARG);
   }
-  const int64_t s_begin = static_cast<int64_t>(split) * p.chunk;
+  // the last CTA of a sink launch reads sink rows j < pos - W + 1 (the rest are in the ring)
+  const bool sink_part = split >= p.splits;
+  int64_t s_begin = static_cast<int64_t>(split) * p.chunk;
   int64_t s_end = s_begin + p.chunk;
   if (s_end > nvalid) s_end = nvalid;
+  if (sink_part) {
+    s_begin = 0;
+    s_end = pos < 0 ? 0 : pos - p.W + 1;
+    if (s_end > p.n_sink) s_end = p.n_sink;
+  }
 
   // q slices of the G heads (8 dims each), pre-scaled into the base-2 domain
   float2 qv[G][4];
@@ -111,9 +125,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const Deco
     for (int i = 0; i < 4; ++i) qv[g][i] = make_float2(f[i].x * p.scale_log2, f[i].y * p.scale_log2);
   }
 
-  const int64_t kv_base = (static_cast<int64_t>(b) * p.Hkv + kvh) * p.W;
-  const __nv_bfloat16 *kbase = p.k_ring + kv_base * D + sub * 8;
-  const __nv_bfloat16 *vbase = p.v_ring + kv_base * D + sub * 8;
+  const int64_t kv_base = (static_cast<int64_t>(b) * p.Hkv + kvh) * (sink_part ? p.n_sink : p.W);
+  const __nv_bfloat16 *kbase = (sink_part ? p.k_sink : p.k_ring) + kv_base * D + sub * 8;
+  const __nv_bfloat16 *vbase = (sink_part ? p.v_sink : p.v_ring) + kv_base * D + sub * 8;
 
   float2 o[G][4];
 #pragma unroll
@@ -268,7 +282,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(const Deco
         L = fmaf(s_l[w][g], wt, L);
       }
     }
-    const int64_t row = (static_cast<int64_t>(b) * p.H + kvh * G + g) * p.splits + split;
+    const int64_t row = (static_cast<int64_t>(b) * p.H + kvh * G + g) * p.n_part + split;
     p.ws_o[row * D + c] = acc;
     if (c == 0) {
       p.ws_ml[row * 2 + 0] = M;
@@ -284,16 +298,16 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t bh = blockIdx.x;
   const int c = threadIdx.x;
-  const float *ml = p.ws_ml + bh * p.splits * 2;
+  const float *ml = p.ws_ml + bh * p.n_part * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, ml[2 * s]);
+  for (int s = 0; s < p.n_part; ++s) M = fmaxf(M, ml[2 * s]);
   float acc = 0.f, L = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < p.splits; ++s) {
+    for (int s = 0; s < p.n_part; ++s) {
       const float m = ml[2 * s];
       if (m == -INFINITY) continue;
       const float wt = ex2(m - M);
-      acc = fmaf(p.ws_o[(bh * p.splits + s) * D + c], wt, acc);
+      acc = fmaf(p.ws_o[(bh * p.n_part + s) * D + c], wt, acc);
       L = fmaf(ml[2 * s + 1], wt, L);
     }
   }

@@ -57,19 +57,26 @@ constexpr float kLazyRescaleLog2 = 8.0f;
 constexpr int kEmuCols = SWA_EMU_COLS;
 static_assert(kEmuCols % 16 == 0 && kEmuCols <= 128, "emulated columns in groups of 16");
 
+// MODE 0: linear [B, heads, N, D] layout.  MODE 1: chunk [B, heads, Tq, D] over
+// a ring [B, Hkv, W, D].  MODE 2: packed token-major [total, heads, D], sequence b
+// on tokens cu_seqlens[b] .. cu_seqlens[b + 1] - 1 (positions from 0 in each).
 struct Fwd2Params {
-  __nv_bfloat16 *out;      // [B, H, n_q, D]
-  float *lse;              // [B, H, n_q] or nullptr
-  const int64_t *q_start;  // MODE 1: [B]
-  int B, H, Hkv, G;
-  int n_q;                 // query rows per (b, h)
-  int n_k;                 // rows of the main key source (N, or Tq for a chunk)
-  int64_t W;               // window (MODE 0: clamped to n_k + kQT)
-  float scale_log2;        // scale * log2(e)
-  int nqt;                 // query tiles per (b, h)
-  int n_ring_tiles;        // MODE 1: ceil(W / kKT)
-  int pair_heads;          // 1: A/B are heads 2p, 2p+1 of a group; 0: q tiles 2p, 2p+1
-  int n_units;
+  __nv_bfloat16 *out = nullptr;        // [B, H, n_q, D]; MODE 2: [total, H, D]
+  float *lse = nullptr;                // [B, H, n_q]; MODE 2: [H, total]; or nullptr
+  const int64_t *q_start = nullptr;    // MODE 1: [B]
+  const int64_t *chunk_len = nullptr;  // MODE 1: [B] valid chunk rows, or nullptr = n_q
+  const int64_t *cu_seqlens = nullptr; // MODE 2: [B + 1]
+  int64_t total = 0;                   // MODE 2: packed tokens
+  int B = 0, H = 0, Hkv = 0, G = 0;
+  int n_q = 0;             // query rows per (b, h); MODE 2: longest sequence
+  int n_k = 0;             // rows of the main key source (N, or Tq for a chunk)
+  int64_t W = 0;           // window (MODE 0 / 2: clamped to n_q + kQT)
+  int n_sink = 0;          // MODE 0 / 2: keys 0 .. n_sink-1 stay visible to later queries
+  float scale_log2 = 0.f;  // scale * log2(e)
+  int nqt = 0;             // query tiles per (b, h)
+  int n_ring_tiles = 0;    // MODE 1: ceil(W / kKT)
+  int pair_heads = 0;      // 1: A/B are heads 2p, 2p+1 of a group; 0: q tiles 2p, 2p+1
+  int n_units = 0;
 };
 
 template <int D>
@@ -130,9 +137,11 @@ __device__ __forceinline__ Unit decode_unit(int u, const Fwd2Params &p) {
 
 // Live key tiles of a unit in stream order, with the class for each query
 // tile.  Positions are int32: MODE 0 uses absolute positions (< 2^30),
-// MODE 1 positions relative to the chunk start (ring slots hold -W .. -1).
-// The segment bases follow the ring layout of swa_tile.cuh.
-template <int MODE>
+// MODE 1 positions relative to the chunk start (ring slots hold -W .. -1),
+// MODE 2 positions within the unit's sequence.  The segment bases follow the
+// ring layout of swa_tile.cuh.  With sinks (SINK, MODE 0 / 2), key tile 0
+// comes first when the window does not reach it.
+template <int MODE, bool SINK>
 struct Walker2 {
   int kt, kt_end;
   int qlo[2], qhi[2];
@@ -143,18 +152,24 @@ struct Walker2 {
   bool full_ring;
   bool has_b;
   int live_a_end, live_b_begin;  // MODE 0: A is live on [kt, live_a_end], B on [live_b_begin, kt_end)
+  int n_sink;        // MODE 0 / 2: sink keys 0 .. n_sink-1
+  bool sink_pending;  // tile 0 (sinks only) still to be yielded ahead of kt
 
-  __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs) {
+  // len: valid query rows of this unit's sequence (MODE 1: also its chunk keys)
+  __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs, int len) {
     has_b = U.has_b;
-    n_k = p.n_k;
+    n_k = MODE == 0 ? p.n_k : len;
     W = static_cast<int>(p.W);
+    n_sink = (SINK && MODE != 1) ? p.n_sink : 0;
+    sink_pending = false;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
       qlo[x] = U.t[x] * kQT;
-      qhi[x] = min(qlo[x] + kQT, p.n_q) - 1;
+      qhi[x] = min(qlo[x] + kQT, len) - 1;
     }
-    if (MODE == 0) {
+    if (MODE != 1) {
       kt = max(qlo[0] - (W - 1), 0) / kKT;
+      sink_pending = SINK && n_sink > 0 && kt > 0;
       kt_end = (has_b ? qhi[1] : qhi[0]) / kKT + 1;
       // the windows of consecutive rows overlap, so each tile's live key tiles are
       // one contiguous range: [first key of its first row, its last row] in tiles
@@ -166,7 +181,7 @@ struct Walker2 {
     } else {
       nrt = p.n_ring_tiles;
       kt = 0;
-      kt_end = nrt + (p.n_q + kKT - 1) / kKT;
+      kt_end = nrt + (len + kKT - 1) / kKT;
       full_ring = qs >= p.W;
       wrap = static_cast<int>(full_ring ? qs % p.W : qs);
     }
@@ -178,7 +193,7 @@ struct Walker2 {
     lo[1] = 1;
     hi[1] = 0;
     base[1] = 0;
-    if (MODE == 0 || k >= nrt) {
+    if (MODE != 1 || k >= nrt) {
       const int c0 = (k - nrt) * kKT;
       const int nc = min(kKT, n_k - c0);
       src = 0;
@@ -224,36 +239,58 @@ struct Walker2 {
   }
 
   // Advance to the next live tile, reporting only which query tiles use it
-  // (ca, cb nonzero) -- what the producer and the MMA issuer need.  MODE 0
-  // reduces to two comparisons per tile; MODE 1 runs the full classification.
+  // (ca, cb nonzero) -- what the producer and the MMA issuer need.  MODE 0 / 2
+  // reduce to two comparisons per tile; MODE 1 runs the full classification.
+  // Every query row sees key 0, so with sinks tile 0 is live for both tiles.
   __device__ __forceinline__ bool next_live(int &k, int &src, int &y0, int &ca, int &cb) {
-    if (MODE == 0) {
+    if (MODE != 1) {
+      src = 0;
+      if (SINK && sink_pending) {
+        sink_pending = false;
+        k = 0;
+        y0 = 0;
+        ca = 1;
+        cb = has_b;
+        return true;
+      }
       if (kt >= kt_end) return false;
       k = kt++;
-      src = 0;
       y0 = k * kKT;
       ca = k <= live_a_end;
-      cb = has_b && k >= live_b_begin;
+      cb = has_b && (k >= live_b_begin || (SINK && k == 0 && n_sink > 0));
       return true;
     }
     return next(k, src, y0, ca, cb);
   }
 
   // Advance to the next live tile: its index, source, first row and classes.
+  // Tile 0 under sinks is partial unless the window alone covers it.
   __device__ __forceinline__ bool next(int &k, int &src, int &y0, int &ca, int &cb) {
+    int lo[2], hi[2], base[2];
+    if (SINK && MODE != 1 && sink_pending) {
+      sink_pending = false;
+      k = 0;
+      segments(0, lo, hi, base, src, y0);
+      ca = 2;
+      cb = has_b ? 2 : 0;
+      return true;
+    }
     while (kt < kt_end) {
       k = kt++;
-      int lo[2], hi[2], base[2];
       const int nc = segments(k, lo, hi, base, src, y0);
       ca = klass(0, nc, lo, hi, base);
       cb = has_b ? klass(1, nc, lo, hi, base) : 0;
+      if (SINK && MODE != 1 && k == 0 && n_sink > 0) {
+        if (ca != 1) ca = 2;
+        if (has_b && cb != 1) cb = 2;
+      }
       if (ca | cb) return true;
     }
     return false;
   }
 };
 
-template <int D, int MODE>
+template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kFwd2Threads, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
@@ -323,13 +360,33 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     return i * P + ((i & 1) ? P - 1 - c : c);
   };
 
-  auto unit_start = [&](const Unit &U, int64_t &qs) -> bool {
+  // 0: run the unit; 1: invalid start position, chunk length or sequence
+  // offsets (skip, flag); 2: the unit's query rows are all padding of a
+  // shorter chunk or sequence (skip).  qs: MODE 1 the chunk's first position,
+  // MODE 2 the sequence's first token.
+  // Every role evaluates it identically, so they skip the same units.
+  auto unit_start = [&](Unit &U, int64_t &qs, int &len) -> int {
     qs = 0;
+    len = p.n_q;
     if (MODE == 1) {
       qs = p.q_start[U.b];
-      if (qs < 0) return false;
+      if (qs < 0) return 1;
+      if (p.chunk_len) {
+        const int64_t l = p.chunk_len[U.b];
+        if (l < 0 || l > p.n_q) return 1;
+        len = static_cast<int>(l);
+      }
+    } else if (MODE == 2) {
+      const int64_t a = p.cu_seqlens[U.b], e = p.cu_seqlens[U.b + 1];
+      if (a < 0 || e < a || e - a > p.n_q || e > p.total) return 1;
+      qs = a;  // first token of the sequence
+      len = static_cast<int>(e - a);
     }
-    return true;
+    if (MODE != 0) {
+      if (U.t[0] * kQT >= len) return 2;
+      if (U.has_b && U.t[1] * kQT >= len) U.has_b = false;
+    }
+    return 0;
   };
 
   if (warp == 0) {
@@ -337,10 +394,12 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     if (lane == 0) {
       int kv_iter = 0, q_iter = 0;
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        const Unit U = decode_unit(u, p);
+        Unit U = decode_unit(u, p);
         int64_t qs;
-        if (!unit_start(U, qs)) {
-          atomicOr(&g_swa_status, SWA_DEV_BADARG);
+        int len;
+        const int ust = unit_start(U, qs, len);
+        if (ust) {
+          if (ust == 1) atomicOr(&g_swa_status, SWA_DEV_BADARG);
           continue;
         }
         if (q_iter > 0 && !mbar_wait(BAR_QE, (q_iter - 1) & 1, abort_flag)) break;
@@ -350,14 +409,19 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           if (x == 1 && !U.has_b) break;
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
-            tma_load_3d(sQ[x] + pn * (kQT * 128), &tm_q, BAR_QF, pn * 64, U.t[x] * kQT,
-                        U.b * p.H + U.h[x]);
+            if (MODE == 2)
+              tma_load_3d(sQ[x] + pn * (kQT * 128), &tm_q, BAR_QF, pn * 64, U.h[x],
+                          static_cast<int>(qs) + U.t[x] * kQT);
+            else
+              tma_load_3d(sQ[x] + pn * (kQT * 128), &tm_q, BAR_QF, pn * 64, U.t[x] * kQT,
+                          U.b * p.H + U.h[x]);
         }
         ++q_iter;
-        Walker2<MODE> wk;
-        wk.init(U, p, qs);
+        Walker2<MODE, SINK> wk;
+        wk.init(U, p, qs, len);
         int k, src, y0, ca, cb;
-        const int z = U.b * p.Hkv + U.kvh;
+        // MODE 2 maps are {D, heads, tokens}: (head, token) replace (row, plane)
+        const int z = MODE == 2 ? static_cast<int>(qs) : U.b * p.Hkv + U.kvh;
         while (wk.next_live(k, src, y0, ca, cb)) {
           const int sk = kv_iter % NK, sv = kv_iter % NV;
           const CUtensorMap *mk = src == 1 ? &tm_kr : &tm_k;
@@ -368,14 +432,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sK + sk * L::KV_BYTES + pn * (kKT * 128), mk, BAR_KF + 8 * sk, pn * 64,
-                        y0, z);
+                        MODE == 2 ? U.kvh : y0, MODE == 2 ? z + y0 : z);
           if (kv_iter >= NV && !mbar_wait(BAR_VE + 8 * sv, ((kv_iter / NV) - 1) & 1, abort_flag))
             break;
           mbar_expect_tx(BAR_VF + 8 * sv, L::KV_BYTES);
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sV + sv * L::KV_BYTES + pn * (kKT * 128), mv, BAR_VF + 8 * sv, pn * 64,
-                        y0, z);
+                        MODE == 2 ? U.kvh : y0, MODE == 2 ? z + y0 : z);
           ++kv_iter;
         }
         if (*abort_flag) break;
@@ -408,13 +472,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                  idO, (acc || kk > 0) ? 1u : 0u);
       };
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        const Unit U = decode_unit(u, p);
+        Unit U = decode_unit(u, p);
         int64_t qs;
-        if (!unit_start(U, qs)) continue;
+        int len;
+        if (unit_start(U, qs, len)) continue;
         mbar_wait(BAR_QF, q_iter & 1, abort_flag);
         tc_fence_after();
-        Walker2<MODE> wk;
-        wk.init(U, p, qs);
+        Walker2<MODE, SINK> wk;
+        wk.init(U, p, qs, len);
         int k, src, y0, ca, cb, na = 0, nb = 0;
         bool have = wk.next_live(k, src, y0, ca, cb);
         bool first[2] = {true, true};
@@ -434,7 +499,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         // tile B starting one tile after A (query tiles 2p, 2p+1): issue its first
         // S now instead of behind A's first softmax
         bool b_ahead = false;
-        if (MODE == 0 && has_next && nb && !cb) {
+        if (MODE != 1 && has_next && nb && !cb) {
           const int sk1 = (kv_iter + 1) % NK;
           mbar_wait(BAR_KF + 8 * sk1, ((kv_iter + 1) / NK) & 1, abort_flag);
           tc_fence_after();
@@ -443,6 +508,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         }
         tc_commit(BAR_KE + 8 * (kv_iter % NK));  // K(first) is read by both S MMAs
         bool o_done[2] = {false, false};
+        const bool b_contig = MODE != 1 && (!SINK || p.n_sink == 0 || p.pair_heads);
         while (have) {
           if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
           const int sv = kv_iter % NV;
@@ -455,7 +521,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             issue_pv(0, sv, !first[0]);
             first[0] = false;
             // linear keys: a query tile's live tiles are contiguous, so it is done
-            if (MODE == 0 && !(has_next && na)) {
+            // (tile A's stay so with the sink tile in front; B's need not)
+            if (MODE != 1 && !(has_next && na)) {
               tc_commit(BAR_O);
               o_done[0] = true;
             }
@@ -471,7 +538,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             tc_fence_after();
             issue_pv(1, sv, !first[1]);
             first[1] = false;
-            if (MODE == 0 && !(has_next && nb)) {
+            if (b_contig && !(has_next && nb)) {
               tc_commit(BAR_O + 8);
               o_done[1] = true;
             }
@@ -506,12 +573,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     const uint32_t tO = tmem + 256 + x * D + lane_off;
     uint32_t s_cnt = 0, u_iter = 0;
     for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-      const Unit U = decode_unit(u, p);
+      Unit U = decode_unit(u, p);
       int64_t qs;
-      if (!unit_start(U, qs)) continue;
-      Walker2<MODE> wk;
-      wk.init(U, p, qs);
-      const int qrow = U.t[x] * kQT + row;  // MODE 0 absolute, MODE 1 relative to q_start
+      int len;
+      if (unit_start(U, qs, len)) continue;
+      Walker2<MODE, SINK> wk;
+      wk.init(U, p, qs, len);
+      // MODE 0 absolute, MODE 1 relative to q_start, MODE 2 within the sequence
+      const int qrow = U.t[x] * kQT + row;
       float m_run = -INFINITY, l_run = 0.f;
       int nt = 0;
       int k, src, y0, ca, cb;
@@ -534,11 +603,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             lo[g] = max(lo[g], qrow - wk.W + 1 - base[g]);
             hi[g] = min(hi[g], qrow - base[g]);
           }
+          // sinks: columns 0 .. n_sink-1 of tile 0, up to the row itself
+          const int sink_hi = (SINK && MODE != 1 && k == 0) ? min(wk.n_sink - 1, qrow) : -1;
           uint32_t mw[kKT / 32];
 #pragma unroll
           for (int w = 0; w < kKT / 32; ++w)
             mw[w] = range_bits(lo[0] - 32 * w, hi[0] - 32 * w) |
-                    range_bits(lo[1] - 32 * w, hi[1] - 32 * w);
+                    range_bits(lo[1] - 32 * w, hi[1] - 32 * w) |
+                    range_bits(-32 * w, sink_hi - 32 * w);
 #pragma unroll
           for (int c = 0; c < kKT; ++c) s[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
         }
@@ -645,12 +717,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         const float inv_l = 1.f / l_run;
         const int hh = U.h[x];
         __nv_bfloat16 *orow =
-            p.out + (static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow) * static_cast<int64_t>(D);
+            p.out + (MODE == 2 ? (qs + qrow) * p.H + hh
+                               : static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow) *
+                        static_cast<int64_t>(D);
 #pragma unroll
         for (int cb2 = 0; cb2 < D / 32; ++cb2) {
           uint32_t o32[32];
           tmem_ld32(tO + cb2 * 32, o32);
-          if (qrow < p.n_q) {
+          if (qrow < len) {
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
               uint4 v;
@@ -662,8 +736,9 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             }
           }
         }
-        if (p.lse && qrow < p.n_q)
-          p.lse[static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow] =
+        if (p.lse && qrow < len)
+          p.lse[MODE == 2 ? static_cast<int64_t>(hh) * p.total + qs + qrow
+                          : static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow] =
               (m_run + __log2f(l_run)) * 0.6931471805599453f;
       }
       tc_fence_before();

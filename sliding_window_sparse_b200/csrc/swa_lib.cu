@@ -64,6 +64,25 @@ int make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t plan
   return r == CUDA_SUCCESS ? SWA_OK : SWA_ERR_CUDA;
 }
 
+// Token-major packed tensor [total, heads, d]: dims {d, heads, total}, box
+// {64, 1, box_rows} -- the same 128-byte-row swizzled tile in shared memory as
+// make_map's {64, box_rows, 1} box.
+int make_map_tokens(CUtensorMap *m, const void *base, int d, int64_t heads, int64_t total,
+                    int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return SWA_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(total)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(heads)};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : SWA_ERR_CUDA;
+}
+
 inline int check_launch() {
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
@@ -78,12 +97,12 @@ int common_checks(int B, int H, int Hkv, int d, int64_t W, float scale) {
   return SWA_OK;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool SINK = false>
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                const CUtensorMap &tkr, const CUtensorMap &tvr, swa::Fwd2Params p,
                cudaStream_t st) {
   using L = swa::Fwd2Layout<D>;
-  auto kern = swa::fwd2_kernel<D, MODE>;
+  auto kern = swa::fwd2_kernel<D, MODE, SINK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
       cudaSuccess)
     return SWA_ERR_CUDA;
@@ -112,7 +131,7 @@ void decode_split(int B, int Hkv, int64_t W, int *chunk, int *splits) {
 
 template <int D, int G>
 int launch_decode(const swa::DecodeParams &p, cudaStream_t st) {
-  dim3 grid(p.splits, p.Hkv, p.B);
+  dim3 grid(p.n_part, p.Hkv, p.B);
   swa::decode_split_kernel<D, G><<<grid, swa::kDecWarps * 32, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
   // The merge kernel is launched as a programmatic dependent of the split
@@ -196,13 +215,15 @@ int swa_block_meta(int key_mode, int B, int64_t n_q, int64_t n_k, const int64_t 
   return check_launch();
 }
 
-int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
-                 int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream) {
+namespace {
+int attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+             int Hkv, int64_t N, int d, int64_t W, int n_sink, float scale, void *stream) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
   if (N < 1 || N >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_sink > kBK) return SWA_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv;
   if ((e = make_map(&tq, q, d, N, static_cast<int64_t>(B) * H, kBQ))) return e;
   if ((e = make_map(&tk, k, d, N, static_cast<int64_t>(B) * Hkv, kBK))) return e;
@@ -210,7 +231,6 @@ int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
   swa::Fwd2Params p;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
-  p.q_start = nullptr;
   p.B = B;
   p.H = H;
   p.Hkv = Hkv;
@@ -218,17 +238,71 @@ int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
   p.n_q = static_cast<int>(N);
   p.n_k = static_cast<int>(N);
   p.W = W < N + kBQ ? W : N + kBQ;
+  p.n_sink = n_sink;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.nqt = static_cast<int>((N + kBQ - 1) / kBQ);
-  p.n_ring_tiles = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_sink > 0)
+    return d == 128 ? launch_fwd<128, 0, true>(tq, tk, tv, tk, tv, p, st)
+                    : launch_fwd<64, 0, true>(tq, tk, tv, tk, tv, p, st);
   return d == 128 ? launch_fwd<128, 0>(tq, tk, tv, tk, tv, p, st)
                   : launch_fwd<64, 0>(tq, tk, tv, tk, tv, p, st);
 }
+}  // namespace
 
-int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_ring,
-                   const int64_t *q_start, int B, int Hkv, int64_t T, int d, int64_t W,
-                   void *stream) {
+int swa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                 int H, int Hkv, int64_t N, int d, int64_t W, float scale, void *stream) {
+  return attn_fwd(q, k, v, out, lse, B, H, Hkv, N, d, W, 0, scale, stream);
+}
+
+int swa_attn_fwd_sink(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                      int H, int Hkv, int64_t N, int d, int64_t W, int n_sink, float scale,
+                      void *stream) {
+  return attn_fwd(q, k, v, out, lse, B, H, Hkv, N, d, W, n_sink, scale, stream);
+}
+
+int swa_attn_varlen(const void *q, const void *k, const void *v, const int64_t *cu_seqlens,
+                    void *out, float *lse, int n_seq, int64_t total, int64_t max_seqlen, int H,
+                    int Hkv, int d, int64_t W, int n_sink, float scale, void *stream) {
+  int e = common_checks(n_seq, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k || !v || !cu_seqlens || !out) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
+  // token coordinates of the tensor maps are int32
+  if (total < 1 || total >= (int64_t(1) << 31) - 2 * kBQ) return SWA_ERR_INVALID_ARG;
+  if (max_seqlen < 1 || max_seqlen >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_sink > kBK) return SWA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if ((e = make_map_tokens(&tq, q, d, H, total, kBQ))) return e;
+  if ((e = make_map_tokens(&tk, k, d, Hkv, total, kBK))) return e;
+  if ((e = make_map_tokens(&tv, v, d, Hkv, total, kBK))) return e;
+  swa::Fwd2Params p;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
+  p.B = n_seq;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.n_q = static_cast<int>(max_seqlen);
+  p.n_k = static_cast<int>(max_seqlen);
+  p.W = W < max_seqlen + kBQ ? W : max_seqlen + kBQ;
+  p.n_sink = n_sink;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nqt = static_cast<int>((max_seqlen + kBQ - 1) / kBQ);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_sink > 0)
+    return d == 128 ? launch_fwd<128, 2, true>(tq, tk, tv, tk, tv, p, st)
+                    : launch_fwd<64, 2, true>(tq, tk, tv, tk, tv, p, st);
+  return d == 128 ? launch_fwd<128, 2>(tq, tk, tv, tk, tv, p, st)
+                  : launch_fwd<64, 2>(tq, tk, tv, tk, tv, p, st);
+}
+
+namespace {
+int ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_ring,
+               const int64_t *q_start, const int64_t *lens, int B, int Hkv, int64_t T, int d,
+               int64_t W, void *stream) {
   if (!k_new || !v_new || !k_ring || !v_ring || !q_start) return SWA_ERR_INVALID_ARG;
   if (B < 1 || Hkv < 1 || T < 1 || W < 1 || (d != 64 && d != 128)) return SWA_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) || !aligned16(v_ring))
@@ -241,14 +315,23 @@ int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_r
   swa::ring_write_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                            static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
-      static_cast<uint4 *>(k_ring), static_cast<uint4 *>(v_ring), q_start, B, Hkv, T, vec, W);
+      static_cast<uint4 *>(k_ring), static_cast<uint4 *>(v_ring), q_start, lens, B, Hkv, T, vec,
+      W);
   return check_launch();
 }
+}  // namespace
 
-int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,
-                        void *v_ring, const int64_t *q_start, void *out, float *lse, int B,
-                        int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
-                        int update_ring, void *stream) {
+int swa_ring_write(const void *k_new, const void *v_new, void *k_ring, void *v_ring,
+                   const int64_t *q_start, int B, int Hkv, int64_t T, int d, int64_t W,
+                   void *stream) {
+  return ring_write(k_new, v_new, k_ring, v_ring, q_start, nullptr, B, Hkv, T, d, W, stream);
+}
+
+namespace {
+int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring, void *v_ring,
+               const int64_t *q_start, const int64_t *chunk_len, void *out, float *lse, int B,
+               int H, int Hkv, int64_t Tq, int d, int64_t W, float scale, int update_ring,
+               void *stream) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k_new || !v_new || !k_ring || !v_ring || !q_start || !out) return SWA_ERR_INVALID_ARG;
@@ -266,6 +349,7 @@ int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, voi
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
   p.q_start = q_start;
+  p.chunk_len = chunk_len;
   p.B = B;
   p.H = H;
   p.Hkv = Hkv;
@@ -280,25 +364,51 @@ int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, voi
   e = d == 128 ? launch_fwd<128, 1>(tq, tk, tv, tkr, tvr, p, st)
                : launch_fwd<64, 1>(tq, tk, tv, tkr, tvr, p, st);
   if (e || !update_ring) return e;
-  return swa_ring_write(k_new, v_new, k_ring, v_ring, q_start, B, Hkv, Tq, d, W, stream);
+  return ring_write(k_new, v_new, k_ring, v_ring, q_start, chunk_len, B, Hkv, Tq, d, W, stream);
+}
+}  // namespace
+
+int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring,
+                        void *v_ring, const int64_t *q_start, void *out, float *lse, int B,
+                        int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                        int update_ring, void *stream) {
+  return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, nullptr, out, lse, B, H, Hkv, Tq, d,
+                    W, scale, update_ring, stream);
+}
+
+int swa_attn_chunk_ring_ragged(const void *q, const void *k_new, const void *v_new,
+                               void *k_ring, void *v_ring, const int64_t *q_start,
+                               const int64_t *chunk_len, void *out, float *lse, int B, int H,
+                               int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                               int update_ring, void *stream) {
+  if (!chunk_len) return SWA_ERR_INVALID_ARG;
+  return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, chunk_len, out, lse, B, H, Hkv, Tq,
+                    d, W, scale, update_ring, stream);
 }
 
 size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int64_t W) {
   if (B < 1 || H < 1 || Hkv < 1 || W < 1 || d < 1) return 0;
   int chunk, splits;
   decode_split(B, Hkv, W, &chunk, &splits);
-  const size_t rows = static_cast<size_t>(B) * H * splits;
+  // one partial per split, plus one for the sink rows of swa_attn_decode_ring_sink
+  const size_t rows = static_cast<size_t>(B) * H * (splits + 1);
   return align256(rows * d * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
-int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
-                         const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
-                         int d, int64_t W, float scale, void *workspace,
-                         size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+int decode_ring(const void *q, const void *k_ring, const void *v_ring, const void *k_sink,
+                const void *v_sink, int n_sink, const int64_t *pos, void *out, float *lse, int B,
+                int H, int Hkv, int d, int64_t W, float scale, void *workspace,
+                size_t workspace_bytes, void *stream) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k_ring || !v_ring || !pos || !out) return SWA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out))
+    return SWA_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_sink > 128) return SWA_ERR_INVALID_ARG;
+  if (n_sink > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink)))
     return SWA_ERR_INVALID_ARG;
   if (W >= (int64_t(1) << 31) || B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
   const size_t need = swa_decode_workspace_bytes(B, H, Hkv, d, W);
@@ -307,6 +417,9 @@ int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
   p.q = static_cast<const __nv_bfloat16 *>(q);
   p.k_ring = static_cast<const __nv_bfloat16 *>(k_ring);
   p.v_ring = static_cast<const __nv_bfloat16 *>(v_ring);
+  p.k_sink = static_cast<const __nv_bfloat16 *>(k_sink);
+  p.v_sink = static_cast<const __nv_bfloat16 *>(v_sink);
+  p.n_sink = n_sink;
   p.pos = pos;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
@@ -315,7 +428,8 @@ int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
   p.Hkv = Hkv;
   p.W = W;
   decode_split(B, Hkv, W, &p.chunk, &p.splits);
-  const size_t rows = static_cast<size_t>(B) * H * p.splits;
+  p.n_part = p.splits + (n_sink > 0 ? 1 : 0);
+  const size_t rows = static_cast<size_t>(B) * H * (p.splits + 1);
   p.ws_o = static_cast<float *>(workspace);
   p.ws_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                       align256(rows * d * sizeof(float)));
@@ -323,6 +437,27 @@ int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = H / Hkv;
   return d == 128 ? dispatch_decode_g<128>(G, p, st) : dispatch_decode_g<64>(G, p, st);
+}
+}  // namespace
+
+extern "C" {
+
+int swa_attn_decode_ring(const void *q, const void *k_ring, const void *v_ring,
+                         const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
+                         int d, int64_t W, float scale, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+  return decode_ring(q, k_ring, v_ring, nullptr, nullptr, 0, pos, out, lse, B, H, Hkv, d, W,
+                     scale, workspace, workspace_bytes, stream);
+}
+
+int swa_attn_decode_ring_sink(const void *q, const void *k_ring, const void *v_ring,
+                              const void *k_sink, const void *v_sink, int n_sink,
+                              const int64_t *pos, void *out, float *lse, int B, int H, int Hkv,
+                              int d, int64_t W, float scale, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+  if (n_sink < 1) return SWA_ERR_INVALID_ARG;
+  return decode_ring(q, k_ring, v_ring, k_sink, v_sink, n_sink, pos, out, lse, B, H, Hkv, d, W,
+                     scale, workspace, workspace_bytes, stream);
 }
 
 int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,

@@ -95,13 +95,16 @@ __global__ void ring_positions_kernel(int B, const int64_t *__restrict__ n_writt
   slot_pos[idx] = s <= L - 1 ? (L - 1) - ((L - 1 - s) % W) : -1;
 }
 
-// Copy chunk rows t >= T - W (positions start + t among the last W) to slot
-// (start + t) mod W.  One thread moves 16 bytes; d * 2 / 16 threads per row.
+// Copy chunk rows t >= T_b - W (positions start + t among the last W) to slot
+// (start + t) mod W, where T_b = lens[b] (or T when lens is null) is the
+// number of valid rows of sequence b.  One thread moves 16 bytes;
+// d * 2 / 16 threads per row.
 __global__ void ring_write_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                                   uint4 *__restrict__ k_ring, uint4 *__restrict__ v_ring,
-                                  const int64_t *__restrict__ q_start, int B, int Hkv, int64_t T,
+                                  const int64_t *__restrict__ q_start,
+                                  const int64_t *__restrict__ lens, int B, int Hkv, int64_t T,
                                   int vec_per_row, int64_t W) {
-  const int64_t rows = T < W ? T : W;  // rows written per (b, kvh)
+  const int64_t rows = T < W ? T : W;  // row slots per (b, kvh)
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total = static_cast<int64_t>(B) * Hkv * rows * vec_per_row;
   if (idx >= total) return;
@@ -110,11 +113,14 @@ __global__ void ring_write_kernel(const uint4 *__restrict__ k_new, const uint4 *
   const int64_t bh = idx / (static_cast<int64_t>(vec_per_row) * rows);
   const int64_t b = bh / Hkv;
   const int64_t start = q_start[b];
-  if (start < 0) {
+  const int64_t tb = lens ? lens[b] : T;
+  if (start < 0 || tb < 0 || tb > T) {
     if (c == 0 && r == 0) atomicOr(&g_swa_status, SWA_DEV_BADARG);
     return;
   }
-  const int64_t t = T - rows + r;  // chunk row
+  const int64_t rows_b = tb < W ? tb : W;
+  if (r >= rows_b) return;
+  const int64_t t = tb - rows_b + r;  // chunk row
   const int64_t slot = (start + t) % W;
   const uint4 kv = k_new[(bh * T + t) * vec_per_row + c];
   const uint4 vv = v_new[(bh * T + t) * vec_per_row + c];

@@ -49,6 +49,9 @@ STREAM = {
     "v_new": 7,
     "ctx_len": 8,
     "extra": 9,
+    "seq_len": 10,
+    "k_sink": 11,
+    "v_sink": 12,
 }
 
 

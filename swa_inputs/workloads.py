@@ -1,8 +1,9 @@
 """The synthetic workloads: shapes, seeds and value recipes (no attention arithmetic).
 
 Every tensor is bf16 i.i.d. N(0, 1) from :func:`swa_inputs.normal_bf16` with the
-workload's seed and the tensor's own stream id.  Decode context lengths are
-uniform integers from the same generator.
+workload's seed and the tensor's own stream id.  Decode context lengths, packed
+sequence lengths and ragged chunk lengths are uniform integers from the same
+generator.
 """
 
 from __future__ import annotations
@@ -29,6 +30,10 @@ class Workload:
     q_start: int = 0   # chunk start (same for every sequence)
     ctx_lo: int = 0    # decode context length range (inclusive)
     ctx_hi: int = 0
+    n_sink: int = 0    # attention sinks: positions 0 .. n_sink-1 stay visible
+    n_seq: int = 0     # varlen: sequences in the packed batch
+    len_lo: int = 0    # varlen sequence / ragged chunk length range (inclusive)
+    len_hi: int = 0
     seed: int = 0
     note: str = field(default="", compare=False)
 
@@ -49,7 +54,30 @@ WORKLOADS = {
                            q_start=12288, seed=3, note="chunked prefill on a ring cache"),
     "decode_ring": Workload("decode_ring", "decode", B=64, H=32, Hkv=8, d=128, W=4096,
                             ctx_lo=4096, ctx_hi=131072, seed=4, note="batched decode"),
+    # the next rows: packed variable-length prefill, sinks, ragged chunks
+    "varlen_prefill": Workload("varlen_prefill", "varlen", B=1, H=32, Hkv=8, d=128, W=4096,
+                               n_seq=16, len_lo=256, len_hi=16384, seed=5,
+                               note="16 packed sequences of 256..16384 tokens"),
+    "mistral_prefill_sink": Workload("mistral_prefill_sink", "prefill", B=1, H=32, Hkv=8, d=128,
+                                     W=4096, N=8192, n_sink=4, seed=6,
+                                     note="Mistral-shaped prefill with 4 attention sinks"),
+    "chunk_ring_ragged": Workload("chunk_ring_ragged", "chunk", B=4, H=32, Hkv=8, d=128, W=4096,
+                                  Tq=512, q_start=12288, len_lo=1, len_hi=512, seed=7,
+                                  note="chunks of 1..512 valid rows on a ring cache"),
+    "decode_ring_sink": Workload("decode_ring_sink", "decode", B=64, H=32, Hkv=8, d=128, W=4096,
+                                 ctx_lo=4096, ctx_hi=131072, n_sink=4, seed=8,
+                                 note="batched decode with 4 attention sinks"),
 }
+
+
+def seq_lens(w: Workload) -> np.ndarray:
+    """Packed sequence lengths (varlen) or valid chunk rows per sequence (ragged chunk)."""
+    count = w.n_seq if w.kind == "varlen" else w.B
+    return uniform_int(w.seed, STREAM["seq_len"], count, w.len_lo, w.len_hi)
+
+
+def cu_seqlens(w: Workload) -> np.ndarray:
+    return np.concatenate([[0], np.cumsum(seq_lens(w))]).astype(np.int64)
 
 
 def prefill_inputs(w: Workload):
@@ -57,6 +85,23 @@ def prefill_inputs(w: Workload):
     k = normal_bf16(w.seed, STREAM["k"], (w.B, w.Hkv, w.N, w.d))
     v = normal_bf16(w.seed, STREAM["v"], (w.B, w.Hkv, w.N, w.d))
     return q, k, v
+
+
+def varlen_inputs(w: Workload):
+    """Token-major packed q [total, H, d], k, v [total, Hkv, d] and cu_seqlens."""
+    cu = cu_seqlens(w)
+    total = int(cu[-1])
+    q = normal_bf16(w.seed, STREAM["q"], (total, w.H, w.d))
+    k = normal_bf16(w.seed, STREAM["k"], (total, w.Hkv, w.d))
+    v = normal_bf16(w.seed, STREAM["v"], (total, w.Hkv, w.d))
+    return q, k, v, cu
+
+
+def sink_inputs(w: Workload):
+    """Sink rows [B, Hkv, n_sink, d] of a decode workload."""
+    k = normal_bf16(w.seed, STREAM["k_sink"], (w.B, w.Hkv, w.n_sink, w.d))
+    v = normal_bf16(w.seed, STREAM["v_sink"], (w.B, w.Hkv, w.n_sink, w.d))
+    return k, v
 
 
 def chunk_inputs(w: Workload):

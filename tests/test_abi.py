@@ -28,7 +28,8 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = declared_symbols()
-    for want in ["swa_block_meta", "swa_attn_fwd", "swa_attn_chunk_ring", "swa_attn_decode_ring",
+    for want in ["swa_block_meta", "swa_attn_fwd", "swa_attn_chunk_ring",
+                 "swa_attn_chunk_ring_ragged", "swa_attn_decode_ring",
                  "swa_decode_workspace_bytes", "swa_ring_write", "swa_ring_slot_positions",
                  "swa_get_device_status", "swa_status_string", "swa_version"]:
         assert want in names
@@ -94,6 +95,15 @@ def test_fwd_rejects_null_and_misaligned(native):
     assert lib.swa_attn_fwd(None, FAKE, FAKE, FAKE, None, 1, 4, 4, 128, 64, 16, 0.1, None) == 1
     odd = ctypes.c_void_p(0x100008)
     assert lib.swa_attn_fwd(odd, FAKE, FAKE, FAKE, None, 1, 4, 4, 128, 64, 16, 0.1, None) == 1
+
+
+def test_ragged_chunk_rejects_null_lengths(native):
+    lib = native.lib()
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert lib.swa_attn_chunk_ring_ragged(*args, None, FAKE, None, 1, 4, 4, 128, 64, 64, 0.1, 0,
+                                          None) == 1
+    assert lib.swa_attn_chunk_ring_ragged(*args, FAKE, FAKE, None, 1, 4, 4, 0, 64, 64, 0.1, 0,
+                                          None) == 1
 
 
 def test_decode_rejects_small_workspace(native):

@@ -128,3 +128,88 @@ def test_negative_start_reports_device_error(swa):
     qs = torch.tensor([-1], dtype=torch.int64, device="cuda")
     swa.swa_attn_chunk_ring(z, zk, zk, rk, rk.clone(), qs, 0.1)
     assert swa.swa_get_device_status() == 6
+
+
+def _run_ragged(swa, q, kn, vn, rk, rv, qs, lens, scale, update=False, fill=7.0):
+    tq, tkn, tvn, trk, trv = (to_dev(x) for x in (q, kn, vn, rk, rv))
+    tqs = torch.tensor(qs, dtype=torch.int64, device="cuda")
+    tl = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    out = torch.full_like(tq, fill)
+    lse = torch.full(tq.shape[:3], fill, dtype=torch.float32, device="cuda")
+    swa.swa_attn_chunk_ring_ragged(tq, tkn, tvn, trk, trv, tqs, tl, scale, update_ring=update,
+                                   out=out, lse=lse, return_lse=True)
+    assert swa.swa_get_device_status() == 0
+    return out, lse, trk, trv
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,d,W,starts,lens", [
+    # full, one token, ends one row past a tile, empty
+    (4, 4, 2, 300, 128, 256, [512, 40, 0, 700], [300, 1, 129, 0]),
+    # odd group size (q-tile pairs), chunk longer than the window, mid-tile ends
+    (3, 6, 2, 256, 64, 128, [1000, 3, 129], [200, 256, 65]),
+    # GQA 4:1 with even group (head pairs), lengths either side of a 128-row tile
+    (3, 8, 2, 384, 128, 512, [12288 + 37, 0, 511], [127, 128, 383]),
+])
+def test_ragged_chunks_per_sequence(swa, B, H, Hkv, Tq, d, W, starts, lens):
+    """Each sequence b equals a plain chunk call on its first lens[b] rows (Chapter 10 s10.2)."""
+    seed = 900 + Tq + W
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    scale = 1.0 / math.sqrt(d)
+    out, lse, trk, trv = _run_ragged(swa, q, kn, vn, rk, rv, starts, lens, scale, update=True)
+    got, got_lse = to_f64(out), to_f64(lse)
+    erk, erv = rk.copy(), rv.copy()
+    for b, (qs, n) in enumerate(zip(starts, lens)):
+        # padding rows stay as the caller left them
+        assert np.all(got[b, :, n:] == 7.0)
+        assert np.all(got_lse[b, :, n:] == 7.0)
+        if n == 0:
+            continue
+        sl = (slice(b, b + 1), slice(None), slice(0, n))
+        ref, ref_lse = oracle.swa_chunk(q[sl], kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [qs], W,
+                                        scale, with_lse=True)
+        assert_close(got[b:b + 1, :, :n], ref, what=f"ragged chunk b={b} len={n}")
+        assert np.max(np.abs(got_lse[b:b + 1, :, :n] - ref_lse)) < 1e-3
+        k1, v1 = oracle.ring_update(kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [qs], W)
+        erk[b:b + 1], erv[b:b + 1] = k1, v1
+    assert np.array_equal(to_host_bits(trk), erk)
+    assert np.array_equal(to_host_bits(trv), erv)
+
+
+def test_ragged_full_lengths_match_plain_call(swa):
+    """chunk_len = Tq everywhere is bit-identical to swa_attn_chunk_ring."""
+    B, H, Hkv, Tq, d, W = 2, 8, 2, 320, 128, 256
+    starts = [4096 + 5, 300]
+    seed = 77
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    scale = 1.0 / math.sqrt(d)
+    o1, l1, _, _ = _run(swa, q, kn, vn, rk, rv, starts, scale)
+    o2, l2, _, _ = _run_ragged(swa, q, kn, vn, rk, rv, starts, [Tq] * B, scale)
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+
+
+
+def test_ragged_chunk_workload_sampled_rows(swa):
+    """The benchmarked ragged chunk batch (1..512 valid rows per sequence), sampled rows."""
+    from swa_inputs.workloads import seq_lens
+
+    w = WORKLOADS["chunk_ring_ragged"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    lens = [int(n) for n in seq_lens(w)]
+    out, _, _, _ = _run_ragged(swa, q, kn, vn, rk, rv, list(qs), lens, w.scale)
+    got = to_f64(out)
+    rng = np.random.default_rng(12)
+    for b, n in enumerate(lens):
+        ts = sorted(set(rng.integers(0, n, 40).tolist()) | {0, n - 1, min(127, n - 1)})
+        rows = np.array([(0, int(rng.integers(w.H)), t) for t in ts], dtype=np.int64)
+        sl = (slice(b, b + 1), slice(None), slice(0, n))
+        ref = oracle.swa_chunk(q[sl], kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [int(qs[b])],
+                               w.W, w.scale, rows=rows)
+        assert_close(got[b, rows[:, 1], rows[:, 2]], ref, what=f"ragged chunk workload b={b}")
+        assert np.all(got[b, :, n:] == 7.0)

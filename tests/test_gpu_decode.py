@@ -9,7 +9,7 @@ import torch
 import oracle
 import swa_inputs as si
 from swa_inputs.workloads import WORKLOADS, decode_inputs
-from tests._util import assert_close, to_dev, to_f64
+from tests._util import assert_close, assert_close_bf16out, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -84,3 +84,46 @@ def test_decode_workspace_reuse_and_exact_size(swa):
     assert np.array_equal(a, b)
     ref = oracle.swa_decode(q, rk, rv, [600, 20], W, 0.125)
     assert_close(a, ref)
+
+
+@pytest.mark.parametrize("B,H,Hkv,d,W,S,pos", [
+    (4, 32, 8, 128, 256, 4, [1000, 255, 258, 3]),       # sinks outside, none, some, partial ring
+    (6, 4, 4, 64, 100, 16, [0, 5, 99, 100, 115, 5000]),  # G = 1, sinks entering the window
+    (2, 16, 2, 128, 4096, 128, [4096 + 200, 70000]),    # G = 8, a full sink tile
+    (1, 4, 2, 64, 1, 2, [9]),                           # W = 1: the query's own key plus two sinks
+])
+def test_decode_sink_full(swa, B, H, Hkv, d, W, S, pos):
+    """Ring decode plus sinks (taxonomy page section 3.2) against the oracle.
+
+    Compared with assert_close_bf16out: rows with W = 1 average three values.
+    """
+    seed = 900 + W + S
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, d))
+    rk = si.normal_bf16(seed, si.STREAM["k_ring"], (B, Hkv, W, d))
+    rv = si.normal_bf16(seed, si.STREAM["v_ring"], (B, Hkv, W, d))
+    sk = si.normal_bf16(seed, si.STREAM["k"], (B, Hkv, S, d))
+    sv = si.normal_bf16(seed, si.STREAM["v"], (B, Hkv, S, d))
+    scale = 1.0 / math.sqrt(d)
+    out, lse = swa.swa_attn_decode_ring(to_dev(q), to_dev(rk), to_dev(rv),
+                                        torch.tensor(pos, dtype=torch.int64, device="cuda"),
+                                        scale, return_lse=True, k_sink=to_dev(sk),
+                                        v_sink=to_dev(sv))
+    assert swa.swa_get_device_status() == 0
+    ref, ref_lse = oracle.swa_decode_sink(q, rk, rv, sk, sv, pos, W, scale, with_lse=True)
+    assert_close_bf16out(to_f64(out), ref, what="decode with sinks")
+    assert np.max(np.abs(to_f64(lse) - ref_lse)) < 1e-3
+
+
+def test_decode_sink_workload_all_rows(swa):
+    """The benchmarked decode with 4 sinks: every (b, h) row."""
+    from swa_inputs.workloads import sink_inputs
+
+    w = WORKLOADS["decode_ring_sink"]
+    q, rk, rv, pos = decode_inputs(w)
+    sk, sv = sink_inputs(w)
+    out = swa.swa_attn_decode_ring(to_dev(q), to_dev(rk), to_dev(rv),
+                                   torch.tensor(pos, dtype=torch.int64, device="cuda"), w.scale,
+                                   k_sink=to_dev(sk), v_sink=to_dev(sv))
+    assert swa.swa_get_device_status() == 0
+    ref = oracle.swa_decode_sink(q, rk, rv, sk, sv, pos, w.W, w.scale)
+    assert_close_bf16out(to_f64(out), ref, what="decode sink workload")
