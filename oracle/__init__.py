@@ -27,6 +27,9 @@ Functions and the passages they follow (page title, section):
 * :func:`swa_varlen`      -- blog section 5.2 tip 4 (packed batches, windows per
                              sequence via cu_seqlens), with optional sinks.
 * :func:`swa_decode_sink` -- taxonomy page section 3.2 on top of the ring decode.
+* :func:`swa_backward`    -- M003 note sections 07-08 (Q/K/V gradients under the
+                             same mask); :func:`swa_forward_f64` is the forward
+                             on fp64 inputs that its finite differences use.
 
 All of them are pinned by ``tests/test_oracle_pins.py``.
 """
@@ -103,6 +106,12 @@ def _configure(lib):
     lib.orc_swa_decode_sink.restype = _i64
     lib.orc_swa_decode_sink.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int,
                                         _int, _i64, _i64, _dbl, _ptr, _ptr]
+    lib.orc_swa_forward_f64.restype = _i64
+    lib.orc_swa_forward_f64.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
+                                        _dbl, _ptr]
+    lib.orc_swa_backward.restype = _i64
+    lib.orc_swa_backward.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
+                                     _dbl, _ptr, _ptr, _ptr]
     lib.orc_tile_classes.restype = _int
     lib.orc_tile_classes.argtypes = [_int, _int, _i64, _i64, _ptr, _i64, _int, _int, _ptr,
                                      _ptr]
@@ -219,6 +228,42 @@ def swa_varlen(q, k, v, cu_seqlens, W: int, scale: float, n_sink: int = 0, rows=
         if lse is not None:
             lse = lse.reshape(total, H)
     return (out, lse) if with_lse else out
+
+
+def _f64(a):
+    """bf16 bit patterns (uint16) -> their exact values; float arrays -> float64."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def swa_forward_f64(q, k, v, W: int, scale: float):
+    """swa_forward on fp64 inputs (the function the gradient pins differentiate)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    out = np.empty((B, H, N, d), dtype=np.float64)
+    if _load().orc_swa_forward_f64(_p(q), _p(k), _p(v), B, H, k.shape[1], N, d, W, scale,
+                                   _p(out)):
+        raise ValueError("query rows without a legal key")
+    return out
+
+
+def swa_backward(q, k, v, dout, W: int, scale: float):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the linear prefill, in fp64.
+
+    q, dout: [B,H,N,d]; k, v: [B,Hkv,N,d]; bf16 bits or float arrays.
+    """
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    dq = np.empty((B, H, N, d), dtype=np.float64)
+    dk = np.empty((B, Hkv, N, d), dtype=np.float64)
+    dv = np.empty((B, Hkv, N, d), dtype=np.float64)
+    if _load().orc_swa_backward(_p(q), _p(k), _p(v), _p(dout), B, H, Hkv, N, d, W, scale,
+                                _p(dq), _p(dk), _p(dv)):
+        raise ValueError("query rows without a legal key")
+    return dq, dk, dv
 
 
 def dense_masked(q, k, v, W: int, scale: float):

@@ -13,7 +13,8 @@
  *
  * Sources (page title, section):
  *  [M003]  "AI infra KB M003: weight sparsity vs attention sparsity"
- *          (xuujii.github.io/ai-infra-kb), sections 03-07.
+ *          (xuujii.github.io/ai-infra-kb), sections 03-08 (07-08: outputs and
+ *          Q/K/V gradients checked under the same mask, by finite differences).
  *  [CH10]  "Chapter 10 -- local and sparse attention: SWA and DSA"
  *          (book.ozine.me, LLMs from scratch), sections 10.1, 10.2, 10.3, 10.6.
  *  [BLOG]  "Dense attention vs sparse sliding window attention"
@@ -516,6 +517,130 @@ int64_t orc_swa_decode_sink(const uint16_t *q, const uint16_t *ring_k, const uin
         free(sc);
     }
     free(maps);
+    return bad;
+}
+
+/*
+ * Gradients of the prefill forward ([M003 s07]: check the Q/K/V gradients,
+ * by finite differences, under the same mask as the output; [M003 s08]:
+ * outputs and gradients with the same mask).  For the loss sum(out * dout):
+ *   P_ij  = softmax over the allowed j of scale * <q_i, k_j>
+ *   dP_ij = <dout_i, v_j>,   D_i = sum_j P_ij dP_ij,   dS_ij = P_ij (dP_ij - D_i)
+ *   dq_i  = scale * sum_j dS_ij k_j
+ *   dk_j  = scale * sum_i dS_ij q_i     (summed over the query heads of j's group)
+ *   dv_j  = sum_i P_ij dout_i           (likewise)
+ * q, dout: [B,H,N,d]; k, v: [B,Hkv,N,d], fp64 values (so that finite
+ * differences can move them by less than a bf16 step); positions 0..N-1.
+ * dq: [B,H,N,d], dk, dv: [B,Hkv,N,d] (fp64, overwritten).
+ * Returns the number of query rows with no legal key (0 for valid inputs).
+ */
+int64_t orc_swa_backward(const double *q, const double *k, const double *v,
+                         const double *dout, int B, int H, int Hkv, int64_t N, int d,
+                         int64_t W, double scale, double *dq, double *dk, double *dv)
+{
+    int64_t bad = 0;
+    memset(dq, 0, sizeof(double) * (size_t)(B * H * N * d));
+    memset(dk, 0, sizeof(double) * (size_t)(B * Hkv * N * d));
+    memset(dv, 0, sizeof(double) * (size_t)(B * Hkv * N * d));
+    /* one (b, kv head) per iteration: its dk, dv rows are written by it alone */
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (int64_t bk = 0; bk < (int64_t)B * Hkv; ++bk) {
+        int64_t b = bk / Hkv, kh = bk % Hkv;
+        int64_t cap = N > 0 ? N : 1;
+        double *p = (double *)malloc(sizeof(double) * (size_t)cap);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)cap);
+        for (int64_t h = 0; h < H; ++h) {
+            if (kv_head(h, H, Hkv) != kh) continue;
+            for (int64_t i = 0; i < N; ++i) {
+                const double *qi = q + ((b * H + h) * N + i) * d;
+                const double *gi = dout + ((b * H + h) * N + i) * d;
+                int64_t lo = i - W + 1 < 0 ? 0 : i - W + 1;
+                if (lo > i) { ++bad; continue; }
+                /* softmax weights over the allowed keys lo..i (two passes) */
+                double smax = -INFINITY;
+                for (int64_t j = lo; j <= i; ++j) {
+                    const double *kj = k + ((b * Hkv + kh) * N + j) * d;
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += qi[c] * kj[c];
+                    p[j - lo] = s * scale;
+                    if (p[j - lo] > smax) smax = p[j - lo];
+                }
+                double denom = 0.0;
+                for (int64_t j = lo; j <= i; ++j) {
+                    p[j - lo] = exp(p[j - lo] - smax);
+                    denom += p[j - lo];
+                }
+                double Di = 0.0;
+                for (int64_t j = lo; j <= i; ++j) {
+                    const double *vj = v + ((b * Hkv + kh) * N + j) * d;
+                    p[j - lo] /= denom;
+                    double g = 0.0;
+                    for (int c = 0; c < d; ++c) g += gi[c] * vj[c];
+                    dp[j - lo] = g;
+                    Di += p[j - lo] * g;
+                }
+                double *dqi = dq + ((b * H + h) * N + i) * d;
+                for (int64_t j = lo; j <= i; ++j) {
+                    double ds = p[j - lo] * (dp[j - lo] - Di);
+                    const double *kj = k + ((b * Hkv + kh) * N + j) * d;
+                    double *dkj = dk + ((b * Hkv + kh) * N + j) * d;
+                    double *dvj = dv + ((b * Hkv + kh) * N + j) * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqi[c] += scale * ds * kj[c];
+                        dkj[c] += scale * ds * qi[c];
+                        dvj[c] += p[j - lo] * gi[c];
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+    }
+    return bad;
+}
+
+/*
+ * The prefill forward of orc_swa_forward on fp64 inputs (positions 0..N-1):
+ * the function whose finite differences pin orc_swa_backward.  Same loops:
+ * scores on the allowed pairs, two-pass softmax, weighted sum of values.
+ * q: [B,H,N,d]; k, v: [B,Hkv,N,d]; out: [B,H,N,d].
+ */
+int64_t orc_swa_forward_f64(const double *q, const double *k, const double *v, int B, int H,
+                            int Hkv, int64_t N, int d, int64_t W, double scale, double *out)
+{
+    int64_t bad = 0;
+#pragma omp parallel reduction(+ : bad)
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < (int64_t)B * H * N; ++r) {
+            int64_t i = r % N, h = (r / N) % H, b = r / (N * H);
+            int64_t kh = kv_head(h, H, Hkv);
+            const double *qi = q + r * d;
+            double *o = out + r * d;
+            int64_t lo = i - W + 1 < 0 ? 0 : i - W + 1;
+            if (lo > i) { ++bad; continue; }
+            double smax = -INFINITY;
+            for (int64_t j = lo; j <= i; ++j) {
+                const double *kj = k + ((b * Hkv + kh) * N + j) * d;
+                double s = 0.0;
+                for (int c = 0; c < d; ++c) s += qi[c] * kj[c];
+                sc[j - lo] = s * scale;
+                if (sc[j - lo] > smax) smax = sc[j - lo];
+            }
+            double denom = 0.0;
+            for (int64_t j = lo; j <= i; ++j) {
+                sc[j - lo] = exp(sc[j - lo] - smax);
+                denom += sc[j - lo];
+            }
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int64_t j = lo; j <= i; ++j) {
+                const double *vj = v + ((b * Hkv + kh) * N + j) * d;
+                for (int c = 0; c < d; ++c) o[c] += sc[j - lo] / denom * vj[c];
+            }
+        }
+        free(sc);
+    }
     return bad;
 }
 

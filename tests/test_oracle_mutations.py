@@ -53,6 +53,11 @@ MUTANTS = {
     "decode_sink_row_fixed": ("kr[n] = sink_k + ((b * Hkv + kh) * S + j) * d;",
                               "kr[n] = sink_k + ((b * Hkv + kh) * S + 0) * d;"),
     "decode_sink_window_edge": ("if (j >= p - W + 1) {", "if (j > p - W + 1) {"),
+    "backward_delta_dropped": ("double ds = p[j - lo] * (dp[j - lo] - Di);",
+                               "double ds = p[j - lo] * dp[j - lo];"),
+    "backward_dk_unscaled": ("dkj[c] += scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
+    "backward_dv_from_q": ("dvj[c] += p[j - lo] * gi[c];", "dvj[c] += p[j - lo] * qi[c];"),
+    "backward_dq_from_q": ("dqi[c] += scale * ds * kj[c];", "dqi[c] += scale * ds * qi[c];"),
 }
 
 
@@ -87,6 +92,10 @@ def _pin_suite(golden_dir):
         lambda: pins.test_sink_tokens_influence_and_middle_tokens_do_not(),
         lambda: pins.test_decode_sink_equals_prefill_row(8, 4, 12),
         lambda: pins.test_decode_sink_equals_prefill_row(16, 4, 50),
+        lambda: pins.test_forward_f64_equals_forward(),
+        lambda: pins.test_backward_finite_differences(3),
+        lambda: pins.test_backward_full_window_equals_torch_autograd(1, 4, 2, 37, 16),
+        lambda: pins.test_backward_window_one(),
     ]
 
 

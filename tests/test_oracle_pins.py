@@ -549,6 +549,78 @@ def test_decode_sink_equals_prefill_row(W, S, P):
         assert np.array_equal(dec, plain)
 
 
+# --- gradients (M003 note section 07: finite-difference check of Q/K/V gradients) ----
+
+def _f64_inputs(seed, B, H, Hkv, N, d):
+    q = si.bf16_bits_to_f32(_rand(seed, (B, H, N, d), si.STREAM["q"])).astype(np.float64)
+    k = si.bf16_bits_to_f32(_rand(seed, (B, Hkv, N, d), si.STREAM["k"])).astype(np.float64)
+    v = si.bf16_bits_to_f32(_rand(seed, (B, Hkv, N, d), si.STREAM["v"])).astype(np.float64)
+    g = si.bf16_bits_to_f32(_rand(seed, (B, H, N, d), si.STREAM["extra"])).astype(np.float64)
+    return q, k, v, g
+
+
+def test_forward_f64_equals_forward():
+    """The fp64-input forward is the bf16-input forward on the same values."""
+    qb = _rand(31, (2, 4, 33, 8), si.STREAM["q"])
+    kb = _rand(31, (2, 2, 33, 8), si.STREAM["k"])
+    vb = _rand(31, (2, 2, 33, 8), si.STREAM["v"])
+    for W in (1, 5, 33):
+        assert np.array_equal(oracle.swa_forward_f64(qb, kb, vb, W, 0.3),
+                              oracle.swa_forward(qb, kb, vb, W, 0.3))
+
+
+@pytest.mark.parametrize("W", [1, 3, 7, 25])
+def test_backward_finite_differences(W):
+    """Central differences of L = sum(out * g) match every gradient entry."""
+    B, H, Hkv, N, d, scale = 1, 4, 2, 12, 4, 0.6
+    q, k, v, g = _f64_inputs(32, B, H, Hkv, N, d)
+    dq, dk, dv = oracle.swa_backward(q, k, v, g, W, scale)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(oracle.swa_forward_f64(q_, k_, v_, W, scale) * g))
+
+    h = 1e-5
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            up = loss(q, k, v)
+            x[idx] = old - h
+            dn = loss(q, k, v)
+            x[idx] = old
+            fd[idx] = (up - dn) / (2 * h)
+        assert np.max(np.abs(fd - grad)) < 1e-7, name
+
+
+@pytest.mark.parametrize("B,H,Hkv,N,d", [(1, 4, 2, 37, 16), (2, 2, 2, 20, 8)])
+def test_backward_full_window_equals_torch_autograd(B, H, Hkv, N, d):
+    """W >= N is causal attention: torch autograd through SDPA in fp64."""
+    import torch
+
+    q, k, v, g = _f64_inputs(33, B, H, Hkv, N, d)
+    scale = 1.0 / math.sqrt(d)
+    tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
+                                                           scale=scale, enable_gqa=(H != Hkv))
+    (out * torch.from_numpy(g)).sum().backward()
+    for W in (N, 3 * N):
+        dq, dk, dv = oracle.swa_backward(q, k, v, g, W, scale)
+        assert np.max(np.abs(dq - tq.grad.numpy())) < 1e-12
+        assert np.max(np.abs(dk - tk.grad.numpy())) < 1e-12
+        assert np.max(np.abs(dv - tv.grad.numpy())) < 1e-12
+
+
+def test_backward_window_one():
+    """W = 1: out = v, so dq = dk = 0 and dv sums dout over the group's heads."""
+    B, H, Hkv, N, d = 2, 6, 2, 15, 8
+    q, k, v, g = _f64_inputs(34, B, H, Hkv, N, d)
+    dq, dk, dv = oracle.swa_backward(q, k, v, g, 1, 0.5)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    want = g.reshape(B, Hkv, H // Hkv, N, d).sum(axis=2)
+    assert np.max(np.abs(dv - want)) < 1e-14
+
+
 # --- the generator itself ------------------------------------------------------
 
 def test_generator_reproducible_and_normal():
