@@ -11,8 +11,8 @@ its own independent batch: weak scaling, no data-path collective).
 
 The same run also times the chunked-prefill-on-ring and decode paths (and the
 narrow-window prefill), then the packed variable-length prefill, prefill and
-decode with attention sinks and ragged chunks, each on its own workload, under
-"paths".  It prints one JSON line
+decode with attention sinks, ragged chunks and the backward pass, each on its
+own workload, under "paths".  It prints one JSON line
 on rank 0, and adds the roofline fraction of the timed kernel, a CPU baseline
 (the fp64 oracle on a bounded sample of rows, timed on the host cores), an
 end-to-end figure through the public API with host buffers, and SM clocks
@@ -76,6 +76,9 @@ def useful_flops(w) -> int:
     """4 * d * (visible pairs) * H, summed over the batch."""
     if w.kind == "prefill":
         return 4 * w.d * w.H * w.B * sequence_pairs(w.N, w.W, w.n_sink)
+    if w.kind == "backward":
+        # five matrix products per visible pair (S, dP, dV, dK, dQ) against the forward's two
+        return 10 * w.d * w.H * w.B * sequence_pairs(w.N, w.W)
     if w.kind == "varlen":
         from swa_inputs.workloads import seq_lens
 
@@ -106,6 +109,9 @@ def algorithmic_bytes(w) -> int:
     e = 2
     if w.kind == "prefill":
         return e * w.d * w.B * (2 * w.H * w.N + 2 * w.Hkv * w.N)
+    if w.kind == "backward":
+        # read q, k, v, out, dout (and lse); write dq, dk, dv
+        return e * w.d * w.B * (4 * w.H * w.N + 4 * w.Hkv * w.N) + 4 * w.B * w.H * w.N
     if w.kind == "varlen":
         from swa_inputs.workloads import cu_seqlens
 
@@ -121,7 +127,7 @@ def algorithmic_bytes(w) -> int:
 
 def describe(w) -> str:
     sink = f" sinks{w.n_sink}" if w.n_sink else ""
-    if w.kind == "prefill":
+    if w.kind in ("prefill", "backward"):
         return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} N{w.N} d{w.d} W{w.W}{sink}"
     if w.kind == "varlen":
         return (f"{w.name}: {w.n_seq} packed sequences, lengths U[{w.len_lo},{w.len_hi}], "
@@ -243,6 +249,15 @@ def make_inputs(w, device, seed_offset=0):
     if w.kind == "prefill":
         return {"q": g("q", (w.B, w.H, w.N, w.d)), "k": g("k", (w.B, w.Hkv, w.N, w.d)),
                 "v": g("v", (w.B, w.Hkv, w.N, w.d))}
+    if w.kind == "backward":
+        import sliding_window_sparse_b200 as swa
+
+        x = {"q": g("q", (w.B, w.H, w.N, w.d)), "k": g("k", (w.B, w.Hkv, w.N, w.d)),
+             "v": g("v", (w.B, w.Hkv, w.N, w.d)), "dout": g("extra", (w.B, w.H, w.N, w.d))}
+        # the forward's output and LSE are inputs of the backward (made once, untimed)
+        x["out"], x["lse"] = swa.swa_attn_fwd(x["q"], x["k"], x["v"], w.W, w.scale,
+                                              return_lse=True)
+        return x
     if w.kind == "varlen":
         from swa_inputs.workloads import cu_seqlens
 
@@ -281,6 +296,12 @@ def make_call(w, x, swa):
         out = torch.empty_like(x["q"])
         return (lambda: swa.swa_attn_fwd(x["q"], x["k"], x["v"], w.W, w.scale, out=out,
                                          n_sink=w.n_sink), out, 1)
+    if w.kind == "backward":
+        dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+        ws = torch.empty(int(swa.lib().swa_attn_bwd_workspace_bytes(w.B, w.H, w.N)),
+                         dtype=torch.uint8, device=x["q"].device)
+        return (lambda: swa.swa_attn_bwd(x["q"], x["k"], x["v"], x["out"], x["dout"], x["lse"],
+                                         w.W, w.scale, dq=dq, dk=dk, dv=dv, workspace=ws), dq, 2)
     if w.kind == "varlen":
         from swa_inputs.workloads import seq_lens
 
@@ -506,7 +527,7 @@ def run_native(args):
     if not args.headline_only:
         for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring",
                      "varlen_prefill", "mistral_prefill_sink", "chunk_ring_ragged",
-                     "decode_ring_sink"):
+                     "decode_ring_sink", "mistral_backward"):
             if name == headline:
                 continue
             pw = WORKLOADS[name]

@@ -146,6 +146,36 @@ SWA_API int swa_attn_varlen(const void *q, const void *k, const void *v,
                             int n_sink, float scale, void *stream);
 
 /*
+ * swa_attn_bwd_workspace_bytes -- bytes of scratch swa_attn_bwd needs (one
+ * fp32 D_i = <dout_i, out_i> per query row: B * H * N * 4, 256-aligned).
+ */
+SWA_API size_t swa_attn_bwd_workspace_bytes(int B, int H, int64_t N);
+
+/*
+ * swa_attn_bwd -- gradients of the tile-skipping prefill (swa_attn_fwd).
+ * Passage: M003 note sections 07-08 (outputs and Q/K/V gradients are checked
+ * under the same window mask); the window rule of sections 03-04.
+ * For the loss sum(out * dout), with P the softmax of scale * Q K^T over the
+ * allowed keys: dV = P^T dout, dP = dout V^T, D_i = <dout_i, out_i>,
+ * dS = P o (dP - D), dQ = scale * dS K, dK = scale * dS^T Q; dK and dV are
+ * summed over the G query heads of each KV head.  Key tiles outside every
+ * window of a query tile are skipped, as in the forward.
+ *   q, out, dout: [B, H, N, d] bf16, device (out: the forward's output)
+ *   k, v:         [B, Hkv, N, d] bf16, device
+ *   lse:  [B, H, N] fp32, device: the forward's natural-log LSE (same scale)
+ *   dq:   [B, H, N, d] bf16, device (written)
+ *   dk, dv: [B, Hkv, N, d] bf16, device (written, not accumulated)
+ *   workspace: device scratch of at least swa_attn_bwd_workspace_bytes(B, H,
+ *         N) bytes, caller-owned; contents on entry are ignored.
+ * Two kernels on `stream`: dQ (which also writes D_i), then dK/dV.
+ * Limits as swa_attn_fwd: 1 <= N < 2^29, d in {64, 128}.
+ */
+SWA_API int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out,
+                         const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                         int H, int Hkv, int64_t N, int d, int64_t W, float scale,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * swa_attn_chunk_ring -- chunked prefill over a W-slot ring-buffer KV cache.
  * Passage: Chapter 10 section 10.2 (a chunk of T_q queries needs the union of
  * W + T_q - 1 keys; the persistent cache keeps only the last W); M003 note

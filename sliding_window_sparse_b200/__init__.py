@@ -26,6 +26,7 @@ __all__ = [
     "swa_block_meta",
     "swa_attn_fwd",
     "swa_attn_fwd_sink",
+    "swa_attn_bwd",
     "swa_attn_varlen",
     "swa_attn_chunk_ring",
     "swa_attn_chunk_ring_ragged",
@@ -120,6 +121,37 @@ def swa_attn_fwd(q, k, v, W: int, scale: float | None = None, out=None, lse=None
         check("swa_attn_fwd", lib().swa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                                  B, H, Hkv, N, d, W, scale, _stream(q.device)))
     return (out, lse) if return_lse else out
+
+
+def swa_attn_bwd(q, k, v, out, dout, lse, W: int, scale: float | None = None, dq=None, dk=None,
+                 dv=None, workspace=None):
+    """Gradients of swa_attn_fwd: returns (dq [B,H,N,d], dk, dv [B,Hkv,N,d]).
+
+    out and lse are the forward's output and natural-log LSE; dout is the incoming gradient.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, dims=4)
+    _need(lse, "lse", torch.float32, 3)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, N, d) or tuple(v.shape) != (B, Hkv, N, d):
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    if tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("out and dout must match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = int(lib().swa_attn_bwd_workspace_bytes(B, H, N))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check("swa_attn_bwd",
+          lib().swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d, W, scale,
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(q.device)))
+    return dq, dk, dv
 
 
 def swa_attn_varlen(q, k, v, cu_seqlens, max_seqlen: int, W: int, scale: float | None = None,

@@ -1,0 +1,690 @@
+// swa_bwd.cuh -- gradients of the sliding-window prefill on tcgen05 tensor cores.
+//
+// The M003 note (section 07) checks the Q/K/V gradients of the windowed
+// attention under the same mask as the forward output; the gradients are
+// those of the loss sum(out * dout):
+//   P = softmax over the allowed keys of scale * Q K^T (from the forward's LSE)
+//   dP = dout V^T,  D_i = <dout_i, out_i>,  dS = P o (dP - D)
+//   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dout
+// with dK and dV summed over the G query heads of a KV head.
+//
+// Two persistent kernels, each shaped like the forward: one thread issues the
+// MMAs, one feeds TMA, four warps (one 128-row tile, a row per thread) do the
+// element-wise work between the MMAs in tensor memory.
+//
+//  * bwd_dq_kernel: one query tile of one head per unit.  Per live key tile:
+//    S = Q K^T and dP = dO V^T on the tensor cores, dS = P o (dP - D) in
+//    registers (P from the LSE, no running max), dQ += dS K with dS read from
+//    tensor memory.  It also writes D_i (which it computes from out and dout
+//    rows at the start of the unit) for the second kernel.
+//  * bwd_dkdv_kernel: one key tile of one KV head per unit, walking every
+//    (query head of the group, live query tile): S^T = K Q^T, dP^T = V dO^T,
+//    P^T and dS^T in registers (a row per key), dV += P^T dO and
+//    dK += dS^T Q with P^T, dS^T read from tensor memory.
+//
+// Key tile j and query tile t interact iff some key of j is in the window of
+// some query of t (the M003 note, section 04's skip rule); partial tiles are
+// masked per row with 128-bit column masks.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace swa {
+
+constexpr int kBwdT = 128;            // query and key tile rows
+constexpr int kBwdThreads = 6 * 32;   // producer, MMA issuer, 4 element-wise warps
+
+struct BwdParams {
+  const __nv_bfloat16 *out;   // [B, H, N, D]
+  const __nv_bfloat16 *dout;  // [B, H, N, D]
+  const float *lse;           // [B, H, N] natural log
+  float *delta;               // [B, H, N] workspace: D_i
+  __nv_bfloat16 *dq;          // [B, H, N, D]
+  __nv_bfloat16 *dk, *dv;     // [B, Hkv, N, D]
+  int B = 0, H = 0, Hkv = 0, G = 0;
+  int N = 0;
+  int W = 0;                  // window, clamped to N + kBwdT
+  float scale = 0.f, scale_log2 = 0.f;
+  int nt = 0;                 // tiles per (b, head): ceil(N / 128)
+  int n_units = 0;
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int PANELS = D / 64;
+  static constexpr uint32_t TILE = kBwdT * D * 2;  // one 128-row bf16 tile
+  static constexpr int NS = 2;                      // streamed-tile stages
+  // dq kernel: Q, dO once per unit; K, V per key tile
+  // dkdv kernel: K, V once per unit; Q, dO per step
+  static constexpr uint32_t OFF_A0 = 0;             // Q (dq) / K (dkdv)
+  static constexpr uint32_t OFF_A1 = TILE;          // dO (dq) / V (dkdv)
+  static constexpr uint32_t OFF_S0 = 2 * TILE;      // NS stages of K (dq) / Q (dkdv)
+  static constexpr uint32_t OFF_S1 = OFF_S0 + NS * TILE;  // NS stages of V (dq) / dO (dkdv)
+  static constexpr uint32_t OFF_VEC = OFF_S1 + NS * TILE; // dkdv: lse2 and D per column, 2 copies
+  static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 2 * kBwdT * 4;
+  static constexpr int NBAR = 16 + 4 * NS;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t BYTES = OFF_MISC + 16;
+  static constexpr uint32_t ALLOC = BYTES + 1024;
+};
+
+// Store 16 columns (32x32b.x16, one lane per thread); no wait.
+__device__ __forceinline__ void tmem_st16_b(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Columns [lo, hi] (clipped to the tile) as four 32-bit words.
+__device__ __forceinline__ void col_mask(int lo, int hi, uint32_t (&mw)[4]) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) mw[w] = range_bits(lo - 32 * w, hi - 32 * w);
+}
+
+// ---------------------------------------------------------------------------------- dQ
+// Unit u: (b, h, query tile t), heaviest tiles first.
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + L::OFF_A0, sDO = base + L::OFF_A1;
+  const uint32_t sK = base + L::OFF_S0, sV = base + L::OFF_S1;
+  const uint32_t bar = base + L::OFF_BAR;
+  const uint32_t BAR_QF = bar, BAR_QE = bar + 8;
+  const uint32_t BAR_SF = bar + 16;        // + 8 * S buffer
+  const uint32_t BAR_DPF = bar + 32;
+  const uint32_t BAR_EL = bar + 40;        // element-wise done with tile j (128 arrivals)
+  const uint32_t BAR_DQF = bar + 48;       // dQ final
+  const uint32_t BAR_DQE = bar + 56;       // dQ read out (128 arrivals)
+  const uint32_t BAR_KF = bar + 128;       // + 8 * stage
+  const uint32_t BAR_KE = BAR_KF + 8 * NS;
+  const uint32_t BAR_VF = BAR_KE + 8 * NS;
+  const uint32_t BAR_VE = BAR_VF + 8 * NS;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_QF, 1);
+    mbar_init(BAR_QE, 1);
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_SF + 8, 1);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_EL, 4 * 32);
+    mbar_init(BAR_DQF, 1);
+    mbar_init(BAR_DQE, 4 * 32);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(BAR_KF + 8 * s, 1);
+      mbar_init(BAR_KE + 8 * s, 1);
+      mbar_init(BAR_VF + 8 * s, 1);
+      mbar_init(BAR_VE + 8 * s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // tensor memory: S double buffer [0, 256), dP [256, 384), dQ [384, 384 + D)
+  const uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
+
+  // unit -> (b, h, t); the key tiles of query tile t are [k_lo, t]
+  auto unit = [&](int u, int &b, int &h, int &t, int &k_lo) {
+    const int per_t = p.B * p.H;
+    t = p.nt - 1 - u / per_t;
+    const int bh = u % per_t;
+    b = bh / p.H;
+    h = bh % p.H;
+    k_lo = max(t * kBwdT - (p.W - 1), 0) / kBwdT;
+  };
+  auto unit_of = [&](int i) -> int {
+    const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return i * P + ((i & 1) ? P - 1 - c : c);
+  };
+
+  if (warp == 0) {
+    // --------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int q_iter = 0, kv_iter = 0;
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+        int b, h, t, k_lo;
+        unit(u, b, h, t, k_lo);
+        if (q_iter > 0 && !mbar_wait(BAR_QE, (q_iter - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(BAR_QF, 2 * L::TILE);
+        const int zq = b * p.H + h;
+#pragma unroll
+        for (int pn = 0; pn < L::PANELS; ++pn) {
+          tma_load_3d(sQ + pn * (kBwdT * 128), &tm_q, BAR_QF, pn * 64, t * kBwdT, zq);
+          tma_load_3d(sDO + pn * (kBwdT * 128), &tm_do, BAR_QF, pn * 64, t * kBwdT, zq);
+        }
+        ++q_iter;
+        const int zk = b * p.Hkv + h / p.G;
+        for (int kt = k_lo; kt <= t; ++kt) {
+          const int st = kv_iter % NS;
+          if (kv_iter >= NS && !mbar_wait(BAR_KE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag))
+            break;
+          mbar_expect_tx(BAR_KF + 8 * st, L::TILE);
+#pragma unroll
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_3d(sK + st * L::TILE + pn * (kBwdT * 128), &tm_k, BAR_KF + 8 * st, pn * 64,
+                        kt * kBwdT, zk);
+          if (kv_iter >= NS && !mbar_wait(BAR_VE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag))
+            break;
+          mbar_expect_tx(BAR_VF + 8 * st, L::TILE);
+#pragma unroll
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_3d(sV + st * L::TILE + pn * (kBwdT * 128), &tm_v, BAR_VF + 8 * st, pn * 64,
+                        kt * kBwdT, zk);
+          ++kv_iter;
+        }
+        if (*abort_flag) break;
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBwdT, kBwdT, false);
+      constexpr uint32_t idQ = idesc_bf16_f32(kBwdT, D, true);
+      int q_iter = 0, kv_iter = 0;
+      uint32_t el_cnt = 0;
+      // S or dP = A (128 x D, K-major) * B (128 x D, K-major)^T
+      auto issue_nt = [&](uint32_t dst, uint32_t a, uint32_t b_) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBwdT * 128) + (kk & 3) * 32;
+          mma_ss(tmem + dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b_ + off, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+        int b, h, t, k_lo;
+        unit(u, b, h, t, k_lo);
+        const int n = t - k_lo + 1;
+        if (!mbar_wait(BAR_QF, q_iter & 1, abort_flag)) break;
+        tc_fence_after();
+        const int kv0 = kv_iter;
+        // S(0), dP(0), S(1)
+        {
+          const int st = kv0 % NS;
+          if (!mbar_wait(BAR_KF + 8 * st, (kv0 / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_nt(T_S, sQ, sK + st * L::TILE);
+          tc_commit(BAR_SF);
+          if (!mbar_wait(BAR_VF + 8 * st, (kv0 / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_nt(T_DP, sDO, sV + st * L::TILE);
+          tc_commit(BAR_DPF);
+          tc_commit(BAR_VE + 8 * st);
+          if (n > 1) {
+            const int st1 = (kv0 + 1) % NS;
+            if (!mbar_wait(BAR_KF + 8 * st1, ((kv0 + 1) / NS) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_nt(T_S + 128, sQ, sK + st1 * L::TILE);
+            tc_commit(BAR_SF + 8);
+          }
+        }
+        // the previous unit's dQ must be read out before this unit's first dQ MMA
+        if (q_iter > 0 && !mbar_wait(BAR_DQE, (q_iter - 1) & 1, abort_flag)) break;
+        for (int j = 0; j < n; ++j) {
+          const int kj = kv0 + j;
+          if (!mbar_wait(BAR_EL, el_cnt & 1, abort_flag)) break;
+          ++el_cnt;
+          tc_fence_after();
+          // dQ += dS(j) K(j): dS in the low 64 columns of S buffer j % 2 (bf16 pairs)
+          const uint32_t aS = tmem + T_S + (j & 1) * 128;
+          const uint32_t kst = sK + (kj % NS) * L::TILE;
+#pragma unroll
+          for (int kk = 0; kk < kBwdT / 16; ++kk)
+            mma_ts(tmem + T_DQ, aS + kk * 8, sdesc_sw128(kst + kk * 16 * 128, kBwdT * 128, 1024),
+                   idQ, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(BAR_KE + 8 * (kj % NS));
+          if (j + 1 < n) {
+            const int st = (kj + 1) % NS;
+            if (!mbar_wait(BAR_VF + 8 * st, ((kj + 1) / NS) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_nt(T_DP, sDO, sV + st * L::TILE);
+            tc_commit(BAR_DPF);
+            tc_commit(BAR_VE + 8 * st);
+          }
+          if (j + 2 < n) {
+            const int st = (kj + 2) % NS;
+            if (!mbar_wait(BAR_KF + 8 * st, ((kj + 2) / NS) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_nt(T_S + (j & 1) * 128, sQ, sK + st * L::TILE);
+            tc_commit(BAR_SF + 8 * (j & 1));
+          }
+        }
+        if (*abort_flag) break;
+        kv_iter += n;
+        tc_commit(BAR_QE);
+        tc_commit(BAR_DQF);
+        ++q_iter;
+      }
+    }
+  } else {
+    // --------------------------------------------------------------- element-wise
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    uint32_t s_cnt[2] = {0u, 0u}, dp_cnt = 0, u_iter = 0;
+    for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+      int b, h, t, k_lo;
+      unit(u, b, h, t, k_lo);
+      const int n = t - k_lo + 1;
+      const int qrow = t * kBwdT + row;
+      const bool valid = qrow < p.N;
+      const int64_t r = (static_cast<int64_t>(b) * p.H + h) * p.N + qrow;
+      // D_i = <dout_i, out_i> (fp32), also written for the dK/dV kernel
+      float Di = 0.f, lse2 = INFINITY;
+      if (valid) {
+        const uint4 *po = reinterpret_cast<const uint4 *>(p.out + r * D);
+        const uint4 *pg = reinterpret_cast<const uint4 *>(p.dout + r * D);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 a = po[c], g = pg[c];
+          const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 af = make_float2(__uint_as_float(aw[i] << 16),
+                                          __uint_as_float(aw[i] & 0xFFFF0000u));
+            const float2 gf = make_float2(__uint_as_float(gw[i] << 16),
+                                          __uint_as_float(gw[i] & 0xFFFF0000u));
+            acc = __ffma2_rn(af, gf, acc);
+          }
+        }
+        Di = acc.x + acc.y;
+        p.delta[r] = Di;
+        lse2 = p.lse[r] * 1.4426950408889634f;
+      }
+      for (int j = 0; j < n; ++j) {
+        const int kt = k_lo + j;
+        const int x = j & 1;
+        if (!mbar_wait(BAR_SF + 8 * x, s_cnt[x] & 1, abort_flag)) break;
+        ++s_cnt[x];
+        if (!mbar_wait(BAR_DPF, dp_cnt & 1, abort_flag)) break;
+        ++dp_cnt;
+        tc_fence_after();
+        // allowed key columns of this row: positions in [qrow - W + 1, qrow] and < N
+        const int c0 = kt * kBwdT;
+        const bool full = c0 + kBwdT - 1 <= t * kBwdT && c0 >= t * kBwdT + kBwdT - p.W &&
+                          t * kBwdT + kBwdT <= p.N;
+        uint32_t mw[4];
+        col_mask(qrow - p.W + 1 - c0, min(qrow, p.N - 1) - c0, mw);
+        const uint32_t tS = tmem + T_S + x * 128 + lane_off;
+        const uint32_t tP = tmem + T_DP + lane_off;
+#pragma unroll
+        for (int ch = 0; ch < kBwdT / 32; ++ch) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS + ch * 32, sr);
+          tmem_ld32(tP + ch * 32, dr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float ds2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 2 * i + e;
+              float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -lse2));
+              if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
+              ds2[e] = pr * (__uint_as_float(dr[c]) - Di);
+            }
+            pk[i] = pack_bf16(ds2[0], ds2[1]);
+          }
+          tmem_st16_b(tS + ch * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR_EL);
+      }
+      if (*abort_flag) break;
+      if (!mbar_wait(BAR_DQF, u_iter & 1, abort_flag)) break;
+      ++u_iter;
+      tc_fence_after();
+      __nv_bfloat16 *drow = p.dq + r * D;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t o32[32];
+        tmem_ld32(tmem + T_DQ + lane_off + cb * 32, o32);
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o32[i + 0]) * p.scale, __uint_as_float(o32[i + 1]) * p.scale);
+            v.y = pack_bf16(__uint_as_float(o32[i + 2]) * p.scale, __uint_as_float(o32[i + 3]) * p.scale);
+            v.z = pack_bf16(__uint_as_float(o32[i + 4]) * p.scale, __uint_as_float(o32[i + 5]) * p.scale);
+            v.w = pack_bf16(__uint_as_float(o32[i + 6]) * p.scale, __uint_as_float(o32[i + 7]) * p.scale);
+            *reinterpret_cast<uint4 *>(drow + cb * 32 + i) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR_DQE);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// -------------------------------------------------------------------------------- dK dV
+// Unit u: (b, kv head, key tile kt); steps over (query head g of the group, live
+// query tile t in [kt, t_hi]).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + L::OFF_A0, sV = base + L::OFF_A1;
+  const uint32_t sQ = base + L::OFF_S0, sDO = base + L::OFF_S1;
+  float *vec = reinterpret_cast<float *>(gbase + L::OFF_VEC);  // [2][2][128]: lse2, D
+  const uint32_t bar = base + L::OFF_BAR;
+  const uint32_t BAR_KVF = bar, BAR_KVE = bar + 8;
+  const uint32_t BAR_SF = bar + 16;
+  const uint32_t BAR_DPF = bar + 24;
+  const uint32_t BAR_EL = bar + 32;        // 128 arrivals
+  const uint32_t BAR_AF = bar + 40;        // dK, dV final
+  const uint32_t BAR_AE = bar + 48;        // dK, dV read out (128 arrivals)
+  const uint32_t BAR_VEC = bar + 56;       // a step's lse2 / D columns staged (128 arrivals)
+  const uint32_t BAR_QF = bar + 128;       // + 8 * stage
+  const uint32_t BAR_QE = BAR_QF + 8 * NS;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_KVF, 1);
+    mbar_init(BAR_KVE, 1);
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_EL, 4 * 32);
+    mbar_init(BAR_AF, 1);
+    mbar_init(BAR_AE, 4 * 32);
+    mbar_init(BAR_VEC, 4 * 32);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(BAR_QF + 8 * s, 1);
+      mbar_init(BAR_QE + 8 * s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // tensor memory: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D)
+  const uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+
+  // unit -> (b, kv head, kt); query tiles [kt, t_hi] of each of the G heads
+  auto unit = [&](int u, int &b, int &kvh, int &kt, int &t_hi) {
+    const int per_t = p.B * p.Hkv;
+    kt = u / per_t;
+    const int bk = u % per_t;
+    b = bk / p.Hkv;
+    kvh = bk % p.Hkv;
+    t_hi = min(p.nt - 1, (kt * kBwdT + kBwdT - 1 + p.W - 1) / kBwdT);
+  };
+  auto unit_of = [&](int i) -> int {
+    const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return i * P + ((i & 1) ? P - 1 - c : c);
+  };
+
+  if (warp == 0) {
+    // --------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int u_iter = 0, q_iter = 0;
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+        int b, kvh, kt, t_hi;
+        unit(u, b, kvh, kt, t_hi);
+        if (u_iter > 0 && !mbar_wait(BAR_KVE, (u_iter - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(BAR_KVF, 2 * L::TILE);
+        const int zk = b * p.Hkv + kvh;
+#pragma unroll
+        for (int pn = 0; pn < L::PANELS; ++pn) {
+          tma_load_3d(sK + pn * (kBwdT * 128), &tm_k, BAR_KVF, pn * 64, kt * kBwdT, zk);
+          tma_load_3d(sV + pn * (kBwdT * 128), &tm_v, BAR_KVF, pn * 64, kt * kBwdT, zk);
+        }
+        ++u_iter;
+        for (int g = 0; g < p.G; ++g) {
+          const int zq = b * p.H + kvh * p.G + g;
+          for (int t = kt; t <= t_hi; ++t) {
+            const int st = q_iter % NS;
+            if (q_iter >= NS && !mbar_wait(BAR_QE + 8 * st, ((q_iter / NS) - 1) & 1, abort_flag))
+              break;
+            mbar_expect_tx(BAR_QF + 8 * st, 2 * L::TILE);
+#pragma unroll
+            for (int pn = 0; pn < L::PANELS; ++pn) {
+              tma_load_3d(sQ + st * L::TILE + pn * (kBwdT * 128), &tm_q, BAR_QF + 8 * st, pn * 64,
+                          t * kBwdT, zq);
+              tma_load_3d(sDO + st * L::TILE + pn * (kBwdT * 128), &tm_do, BAR_QF + 8 * st,
+                          pn * 64, t * kBwdT, zq);
+            }
+            ++q_iter;
+          }
+          if (*abort_flag) break;
+        }
+        if (*abort_flag) break;
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBwdT, kBwdT, false);
+      constexpr uint32_t idA = idesc_bf16_f32(kBwdT, D, true);
+      int u_iter = 0, q_iter = 0;
+      uint32_t el_cnt = 0;
+      auto issue_nt = [&](uint32_t dst, uint32_t a, uint32_t b_) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBwdT * 128) + (kk & 3) * 32;
+          mma_ss(tmem + dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b_ + off, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      // dst (+)= A[tmem, 128 x 128 bf16] * B[128 queries x D, MN-major]
+      auto issue_tn = [&](uint32_t dst, uint32_t a_cols, uint32_t b_, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBwdT / 16; ++kk)
+          mma_ts(tmem + dst, tmem + a_cols + kk * 8,
+                 sdesc_sw128(b_ + kk * 16 * 128, kBwdT * 128, 1024), idA,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+        int b, kvh, kt, t_hi;
+        unit(u, b, kvh, kt, t_hi);
+        const int n = p.G * (t_hi - kt + 1);
+        if (!mbar_wait(BAR_KVF, u_iter & 1, abort_flag)) break;
+        tc_fence_after();
+        const int q0 = q_iter;
+        {
+          const int st = q0 % NS;
+          if (!mbar_wait(BAR_QF + 8 * st, (q0 / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_nt(T_S, sK, sQ + st * L::TILE);
+          tc_commit(BAR_SF);
+          issue_nt(T_DP, sV, sDO + st * L::TILE);
+          tc_commit(BAR_DPF);
+        }
+        // the previous unit's dK, dV must be read out before this unit's first dV, dK MMAs
+        if (u_iter > 0 && !mbar_wait(BAR_AE, (u_iter - 1) & 1, abort_flag)) break;
+        for (int s = 0; s < n; ++s) {
+          const int qs = q0 + s;
+          const int st = qs % NS;
+          if (!mbar_wait(BAR_EL, el_cnt & 1, abort_flag)) break;
+          ++el_cnt;
+          tc_fence_after();
+          issue_tn(T_DV, T_S, sDO + st * L::TILE, s > 0);   // dV += P^T dO
+          issue_tn(T_DK, T_DP, sQ + st * L::TILE, s > 0);   // dK += dS^T Q
+          tc_commit(BAR_QE + 8 * st);
+          if (s + 1 < n) {
+            const int st1 = (qs + 1) % NS;
+            if (!mbar_wait(BAR_QF + 8 * st1, ((qs + 1) / NS) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_nt(T_S, sK, sQ + st1 * L::TILE);
+            tc_commit(BAR_SF);
+            issue_nt(T_DP, sV, sDO + st1 * L::TILE);
+            tc_commit(BAR_DPF);
+          }
+        }
+        if (*abort_flag) break;
+        q_iter += n;
+        tc_commit(BAR_KVE);
+        tc_commit(BAR_AF);
+        ++u_iter;
+      }
+    }
+  } else {
+    // --------------------------------------------------------------- element-wise
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;   // key row of the tile
+    const int et = threadIdx.x - 64;    // 0..127: column this thread stages
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    uint32_t s_cnt = 0, u_iter = 0, step = 0;
+    for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+      int b, kvh, kt, t_hi;
+      unit(u, b, kvh, kt, t_hi);
+      const int krow = kt * kBwdT + row;
+      bool stop = false;
+      for (int g = 0; g < p.G && !stop; ++g) {
+        const int h = kvh * p.G + g;
+        const int64_t rbase = (static_cast<int64_t>(b) * p.H + h) * p.N;
+        for (int t = kt; t <= t_hi; ++t, ++step) {
+          // stage lse2 and D of the tile's 128 query columns (two copies alternate;
+          // passing step s's barrier means every thread has finished step s - 1,
+          // so the copy written at step s + 1 is no longer read)
+          float *v2 = vec + (step & 1) * 2 * kBwdT;
+          const int qc = t * kBwdT + et;
+          v2[et] = qc < p.N ? p.lse[rbase + qc] * 1.4426950408889634f : INFINITY;
+          v2[kBwdT + et] = qc < p.N ? p.delta[rbase + qc] : 0.f;
+          mbar_arrive(BAR_VEC);
+          if (!mbar_wait(BAR_VEC, step & 1, abort_flag) ||
+              !mbar_wait(BAR_SF, s_cnt & 1, abort_flag) ||
+              !mbar_wait(BAR_DPF, s_cnt & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          ++s_cnt;
+          tc_fence_after();
+          // allowed query columns of key row krow: i in [krow, krow + W - 1], i < N
+          const int c0 = t * kBwdT;
+          const bool full = kt * kBwdT + kBwdT - 1 <= c0 && c0 + kBwdT - 1 - kt * kBwdT <= p.W - 1 &&
+                            c0 + kBwdT <= p.N;
+          uint32_t mw[4];
+          col_mask(krow - c0, min(krow + p.W - 1, p.N - 1) - c0, mw);
+          const uint32_t tS = tmem + T_S + lane_off;
+          const uint32_t tP = tmem + T_DP + lane_off;
+#pragma unroll
+          for (int ch = 0; ch < kBwdT / 32; ++ch) {
+            uint32_t sr[32], dr[32];
+            tmem_ld32(tS + ch * 32, sr);
+            tmem_ld32(tP + ch * 32, dr);
+            uint32_t pk[16], dk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float pp[2], dd[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int c = 2 * i + e;
+                const int col = ch * 32 + c;
+                float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -v2[col]));
+                if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
+                pp[e] = pr;
+                dd[e] = pr * (__uint_as_float(dr[c]) - v2[kBwdT + col]);
+              }
+              pk[i] = pack_bf16(pp[0], pp[1]);
+              dk[i] = pack_bf16(dd[0], dd[1]);
+            }
+            tmem_st16_b(tS + ch * 16, pk);
+            tmem_st16_b(tP + ch * 16, dk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(BAR_EL);
+        }
+      }
+      if (stop || *abort_flag) break;
+      if (!mbar_wait(BAR_AF, u_iter & 1, abort_flag)) break;
+      ++u_iter;
+      tc_fence_after();
+      const bool valid = krow < p.N;
+      const int64_t r = (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + krow;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16 *drow = (which == 0 ? p.dv : p.dk) + r * D;
+        const float mul = which == 0 ? 1.f : p.scale;
+        const uint32_t src = tmem + (which == 0 ? T_DV : T_DK) + lane_off;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t o32[32];
+          tmem_ld32(src + cb * 32, o32);
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(o32[i + 0]) * mul, __uint_as_float(o32[i + 1]) * mul);
+              v.y = pack_bf16(__uint_as_float(o32[i + 2]) * mul, __uint_as_float(o32[i + 3]) * mul);
+              v.z = pack_bf16(__uint_as_float(o32[i + 4]) * mul, __uint_as_float(o32[i + 5]) * mul);
+              v.w = pack_bf16(__uint_as_float(o32[i + 6]) * mul, __uint_as_float(o32[i + 7]) * mul);
+              *reinterpret_cast<uint4 *>(drow + cb * 32 + i) = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR_AE);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace swa

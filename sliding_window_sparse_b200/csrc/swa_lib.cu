@@ -15,6 +15,7 @@
 
 #include "../../include/swa.h"
 #include "sm100.cuh"
+#include "swa_bwd.cuh"
 #include "swa_decode.cuh"
 #include "swa_fwd2.cuh"
 #include "swa_meta.cuh"
@@ -458,6 +459,84 @@ int swa_attn_decode_ring_sink(const void *q, const void *k_ring, const void *v_r
   if (n_sink < 1) return SWA_ERR_INVALID_ARG;
   return decode_ring(q, k_ring, v_ring, k_sink, v_sink, n_sink, pos, out, lse, B, H, Hkv, d, W,
                      scale, workspace, workspace_bytes, stream);
+}
+
+size_t swa_attn_bwd_workspace_bytes(int B, int H, int64_t N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return align256(static_cast<size_t>(B) * H * static_cast<size_t>(N) * sizeof(float));
+}
+
+}  // extern "C"
+
+namespace {
+template <int D>
+int launch_bwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+               const CUtensorMap &tdo, swa::BwdParams p, cudaStream_t st) {
+  using L = swa::BwdLayout<D>;
+  auto kq = swa::bwd_dq_kernel<D>;
+  auto kkv = swa::bwd_dkdv_kernel<D>;
+  if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
+          cudaSuccess)
+    return SWA_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return SWA_ERR_CUDA;
+  // dQ (and D_i) first: the dK/dV kernel reads D_i
+  const int64_t uq = static_cast<int64_t>(p.B) * p.H * p.nt;
+  const int64_t ukv = static_cast<int64_t>(p.B) * p.Hkv * p.nt;
+  if (uq > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(uq);
+  kq<<<static_cast<int>(uq < sms ? uq : sms), swa::kBwdThreads, L::ALLOC, st>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+  p.n_units = static_cast<int>(ukv);
+  kkv<<<static_cast<int>(ukv < sms ? ukv : sms), swa::kBwdThreads, L::ALLOC, st>>>(tq, tk, tv, tdo,
+                                                                                  p);
+  return check_launch();
+}
+}  // namespace
+
+extern "C" {
+
+int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int64_t N,
+                 int d, int64_t W, float scale, void *workspace, size_t workspace_bytes,
+                 void *stream) {
+  int e = common_checks(B, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SWA_ERR_INVALID_ARG;
+  if (N < 1 || N >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  const size_t need = swa_attn_bwd_workspace_bytes(B, H, N);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SWA_ERR_WORKSPACE;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((e = make_map(&tq, q, d, N, static_cast<int64_t>(B) * H, swa::kBwdT))) return e;
+  if ((e = make_map(&tk, k, d, N, static_cast<int64_t>(B) * Hkv, swa::kBwdT))) return e;
+  if ((e = make_map(&tv, v, d, N, static_cast<int64_t>(B) * Hkv, swa::kBwdT))) return e;
+  if ((e = make_map(&tdo, dout, d, N, static_cast<int64_t>(B) * H, swa::kBwdT))) return e;
+  swa::BwdParams p;
+  p.out = static_cast<const __nv_bfloat16 *>(out);
+  p.dout = static_cast<const __nv_bfloat16 *>(dout);
+  p.lse = lse;
+  p.delta = static_cast<float *>(workspace);
+  p.dq = static_cast<__nv_bfloat16 *>(dq);
+  p.dk = static_cast<__nv_bfloat16 *>(dk);
+  p.dv = static_cast<__nv_bfloat16 *>(dv);
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.N = static_cast<int>(N);
+  p.W = static_cast<int>(W < N + swa::kBwdT ? W : N + swa::kBwdT);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nt = static_cast<int>((N + swa::kBwdT - 1) / swa::kBwdT);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_bwd<128>(tq, tk, tv, tdo, p, st) : launch_bwd<64>(tq, tk, tv, tdo, p, st);
 }
 
 int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,

@@ -67,6 +67,8 @@ WORKLOADS = {
     "decode_ring_sink": Workload("decode_ring_sink", "decode", B=64, H=32, Hkv=8, d=128, W=4096,
                                  ctx_lo=4096, ctx_hi=131072, n_sink=4, seed=8,
                                  note="batched decode with 4 attention sinks"),
+    "mistral_backward": Workload("mistral_backward", "backward", B=1, H=32, Hkv=8, d=128, W=4096,
+                                 N=8192, seed=9, note="gradients of the Mistral-shaped prefill"),
 }
 
 

@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = declared_symbols()
-    for want in ["swa_block_meta", "swa_attn_fwd", "swa_attn_chunk_ring",
+    for want in ["swa_block_meta", "swa_attn_fwd", "swa_attn_bwd", "swa_attn_chunk_ring",
                  "swa_attn_chunk_ring_ragged", "swa_attn_decode_ring",
                  "swa_decode_workspace_bytes", "swa_ring_write", "swa_ring_slot_positions",
                  "swa_get_device_status", "swa_status_string", "swa_version"]:
