@@ -123,6 +123,30 @@ def algorithmic_bytes(w) -> int:
     return decode_kv_bytes(w) + e * w.d * w.B * w.H * 2
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): the workload seed plus the rank."""
+    return rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's figure (the job's time); all ranks get it."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(work_per_rank: float, world: int, ms_per_step: float, unit_div: float) -> float:
+    """Whole-job throughput: every rank's work divided by the slowest rank's time."""
+    return work_per_rank * world / (ms_per_step * 1e-3) / unit_div
+
+
 # ----------------------------------------------------------------------------- helpers
 
 def describe(w) -> str:
@@ -485,12 +509,8 @@ def run_native(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def job_max(x):
+        return max_over_ranks(x, world, dev)
 
     peaks, peak_src = load_peaks()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -501,26 +521,26 @@ def run_native(args):
     # headline (default: the Mistral-shaped prefill), each rank its own batch
     headline = args.workload
     w = WORKLOADS[headline]
-    x = make_inputs(w, dev, seed_offset=rank)
+    x = make_inputs(w, dev, seed_offset=rank_seed_offset(rank))
     call, out, launches_per_step = make_call(w, x, swa)
     times, t0, t1 = time_steps(call, args.steps, args.warmup, flush, barrier)
     if swa.swa_get_device_status() != 0:
         raise SystemExit("device status error during the timed region")
-    total_ms = max_over_ranks(sum(times))
+    total_ms = job_max(sum(times))
     mean_ms = total_ms / args.steps
     if w.kind == "decode":
         work, unit, scale_div, bound, peak = decode_kv_bytes(w), "GB/s", 1e9, "hbm", "hbm_gbs"
     else:
         work, unit, scale_div, bound, peak = useful_flops(w), "TFLOP/s", 1e12, "tensor", "bf16_tflops"
-    value = work * world / (mean_ms * 1e-3) / scale_div
+    value = job_rate(work, world, mean_ms, scale_div)
     kernel_rate = work / (statistics.mean(times) * 1e-3) / scale_div
     clocks = sampler.summary(t0, t1) if sampler else None
 
     # end to end through the public API with host buffers
     e2e_steps = max(3, min(args.steps, 20))
     e2e_ms, h2d, d2h = time_e2e(w, x, swa, e2e_steps, 2)
-    e2e_ms = max_over_ranks(e2e_ms)
-    e2e_value = work * world / (e2e_ms * 1e-3) / scale_div
+    e2e_ms = job_max(e2e_ms)
+    e2e_value = job_rate(work, world, e2e_ms, scale_div)
 
     # the other paths of the hot path, on their own workloads
     paths = {}
@@ -531,11 +551,11 @@ def run_native(args):
             if name == headline:
                 continue
             pw = WORKLOADS[name]
-            px = make_inputs(pw, dev, seed_offset=rank)
+            px = make_inputs(pw, dev, seed_offset=rank_seed_offset(rank))
             pcall, _, nl = make_call(pw, px, swa)
             psteps = max(10, min(args.steps, 200))
             ptimes, _, _ = time_steps(pcall, psteps, max(3, args.warmup), flush, barrier)
-            pms = max_over_ranks(sum(ptimes)) / psteps
+            pms = job_max(sum(ptimes)) / psteps
             entry = {"workload": name, "ms_per_call": pms, "launches_per_call": nl}
             if pw.kind == "decode":
                 gbs = decode_kv_bytes(pw) / (pms * 1e-3) / 1e9
