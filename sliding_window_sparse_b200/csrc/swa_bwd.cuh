@@ -80,6 +80,23 @@ __device__ __forceinline__ void tmem_st16_b(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
+// Issue a 32-column tensor-memory load without waiting; tmem_ld_wait2 waits
+// for every load this thread issued and ties the two destination arrays to
+// the wait, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait2(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]), "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]), "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
+               :
+               : "memory");
+}
+
 // Columns [lo, hi] (clipped to the tile) as four 32-bit words.
 __device__ __forceinline__ void col_mask(int lo, int hi, uint32_t (&mw)[4]) {
 #pragma unroll
@@ -248,6 +265,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // the previous unit's dQ must be read out before this unit's first dQ MMA
         if (q_iter > 0 && !mbar_wait(BAR_DQE, (q_iter - 1) & 1, abort_flag)) break;
+        // per tile j: dS(j) stored -> dQ(j), dP(j+1), S(j+2).  The element-wise warps
+        // compute P(j+1) from S(j+1) (issued a tile earlier) while dQ(j) and dP(j+1)
+        // run.  Each barrier's next phase depends on this thread having passed the
+        // previous one (EL(j+1) needs dP(j+1), issued after the wait for EL(j)).
         for (int j = 0; j < n; ++j) {
           const int kj = kv0 + j;
           if (!mbar_wait(BAR_EL, el_cnt & 1, abort_flag)) break;
@@ -325,8 +346,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int x = j & 1;
         if (!mbar_wait(BAR_SF + 8 * x, s_cnt[x] & 1, abort_flag)) break;
         ++s_cnt[x];
-        if (!mbar_wait(BAR_DPF, dp_cnt & 1, abort_flag)) break;
-        ++dp_cnt;
         tc_fence_after();
         // allowed key columns of this row: positions in [qrow - W + 1, qrow] and < N
         const int c0 = kt * kBwdT;
@@ -336,25 +355,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         col_mask(qrow - p.W + 1 - c0, min(qrow, p.N - 1) - c0, mw);
         const uint32_t tS = tmem + T_S + x * 128 + lane_off;
         const uint32_t tP = tmem + T_DP + lane_off;
+        // phase 1 (needs only S): P in fp32
+        float pf[kBwdT];
+        auto pchunk = [&](int ch, const uint32_t (&sr)[32]) {
 #pragma unroll
-        for (int ch = 0; ch < kBwdT / 32; ++ch) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tS + ch * 32, sr);
-          tmem_ld32(tP + ch * 32, dr);
+          for (int c = 0; c < 32; ++c) {
+            float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -lse2));
+            if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
+            pf[ch * 32 + c] = pr;
+          }
+        };
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_issue(tS, r0);
+          tmem_ld32_issue(tS + 32, r1);
+          tmem_ld_wait2(r0, r1);
+          pchunk(0, r0);
+          tmem_ld32_issue(tS + 64, r0);
+          pchunk(1, r1);
+          tmem_ld32_issue(tS + 96, r1);
+          tmem_ld_wait2(r0, r1);
+          pchunk(2, r0);
+          pchunk(3, r1);
+        }
+        // phase 2: dS = P o (dP - D) as bf16 over the low half of this S buffer;
+        // dP is released as soon as it is read
+        if (!mbar_wait(BAR_DPF, dp_cnt & 1, abort_flag)) break;
+        ++dp_cnt;
+        tc_fence_after();
+        auto dchunk = [&](int ch, const uint32_t (&dr)[32]) {
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float ds2[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = 2 * i + e;
-              float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -lse2));
-              if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
-              ds2[e] = pr * (__uint_as_float(dr[c]) - Di);
-            }
-            pk[i] = pack_bf16(ds2[0], ds2[1]);
-          }
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(pf[ch * 32 + 2 * i] * (__uint_as_float(dr[2 * i]) - Di),
+                              pf[ch * 32 + 2 * i + 1] * (__uint_as_float(dr[2 * i + 1]) - Di));
           tmem_st16_b(tS + ch * 16, pk);
+        };
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_issue(tP, r0);
+          tmem_ld32_issue(tP + 32, r1);
+          tmem_ld_wait2(r0, r1);
+          dchunk(0, r0);
+          tmem_ld32_issue(tP + 64, r0);
+          dchunk(1, r1);
+          tmem_ld32_issue(tP + 96, r1);
+          tmem_ld_wait2(r0, r1);
+          dchunk(2, r0);
+          dchunk(3, r1);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -416,10 +464,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t BAR_KVF = bar, BAR_KVE = bar + 8;
   const uint32_t BAR_SF = bar + 16;
   const uint32_t BAR_DPF = bar + 24;
-  const uint32_t BAR_EL = bar + 32;        // 128 arrivals
+  const uint32_t BAR_PF = bar + 32;        // P^T of the step stored (128 arrivals)
   const uint32_t BAR_AF = bar + 40;        // dK, dV final
   const uint32_t BAR_AE = bar + 48;        // dK, dV read out (128 arrivals)
   const uint32_t BAR_VEC = bar + 56;       // a step's lse2 / D columns staged (128 arrivals)
+  const uint32_t BAR_DSF = bar + 64;       // dS^T of the step stored (128 arrivals)
   const uint32_t BAR_QF = bar + 128;       // + 8 * stage
   const uint32_t BAR_QE = BAR_QF + 8 * NS;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
@@ -431,10 +480,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR_KVE, 1);
     mbar_init(BAR_SF, 1);
     mbar_init(BAR_DPF, 1);
-    mbar_init(BAR_EL, 4 * 32);
+    mbar_init(BAR_PF, 4 * 32);
     mbar_init(BAR_AF, 1);
     mbar_init(BAR_AE, 4 * 32);
     mbar_init(BAR_VEC, 4 * 32);
+    mbar_init(BAR_DSF, 4 * 32);
     for (int s = 0; s < NS; ++s) {
       mbar_init(BAR_QF + 8 * s, 1);
       mbar_init(BAR_QE + 8 * s, 1);
@@ -551,21 +601,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // the previous unit's dK, dV must be read out before this unit's first dV, dK MMAs
         if (u_iter > 0 && !mbar_wait(BAR_AE, (u_iter - 1) & 1, abort_flag)) break;
+        // per step: P^T(s) stored -> dV(s), S^T(s+1); dS^T(s) stored -> dK(s), dP^T(s+1).
+        // S^T(s+1) overwrites P^T(s) and dP^T(s+1) overwrites dS^T(s), each issued
+        // behind the MMA that reads it; the element-wise warps compute P^T(s+1)
+        // while dK(s) and dP^T(s+1) run.
         for (int s = 0; s < n; ++s) {
           const int qs = q0 + s;
           const int st = qs % NS;
-          if (!mbar_wait(BAR_EL, el_cnt & 1, abort_flag)) break;
-          ++el_cnt;
+          const int st1 = (qs + 1) % NS;
+          if (!mbar_wait(BAR_PF, el_cnt & 1, abort_flag)) break;
           tc_fence_after();
           issue_tn(T_DV, T_S, sDO + st * L::TILE, s > 0);   // dV += P^T dO
-          issue_tn(T_DK, T_DP, sQ + st * L::TILE, s > 0);   // dK += dS^T Q
-          tc_commit(BAR_QE + 8 * st);
           if (s + 1 < n) {
-            const int st1 = (qs + 1) % NS;
             if (!mbar_wait(BAR_QF + 8 * st1, ((qs + 1) / NS) & 1, abort_flag)) break;
             tc_fence_after();
             issue_nt(T_S, sK, sQ + st1 * L::TILE);
             tc_commit(BAR_SF);
+          }
+          if (!mbar_wait(BAR_DSF, el_cnt & 1, abort_flag)) break;
+          ++el_cnt;
+          tc_fence_after();
+          issue_tn(T_DK, T_DP, sQ + st * L::TILE, s > 0);   // dK += dS^T Q
+          tc_commit(BAR_QE + 8 * st);
+          if (s + 1 < n) {
             issue_nt(T_DP, sV, sDO + st1 * L::TILE);
             tc_commit(BAR_DPF);
           }
@@ -588,63 +646,118 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int b, kvh, kt, t_hi;
       unit(u, b, kvh, kt, t_hi);
       const int krow = kt * kBwdT + row;
+      const int nqt = t_hi - kt + 1, n = p.G * nqt;
+      // lse2 and D of query column et of step s: (query head g, query tile t)
+      auto col_vals = [&](int s, float &l2, float &dd) {
+        const int g = s / nqt, t = kt + s % nqt;
+        const int64_t rb = (static_cast<int64_t>(b) * p.H + kvh * p.G + g) * p.N;
+        const int qc = t * kBwdT + et;
+        l2 = qc < p.N ? p.lse[rb + qc] * 1.4426950408889634f : INFINITY;
+        dd = qc < p.N ? p.delta[rb + qc] : 0.f;
+      };
+      // stage a step's 128 (lse2, D) column values (two copies alternate).  Step
+      // s + 1 is staged at the end of step s, after this thread's last read of
+      // the copy it overwrites; passing step s's barrier needs every thread's
+      // staging of step s, which each did after finishing step s - 1.
+      auto stage = [&](uint32_t st, float l2, float dd) {
+        float *v2 = vec + (st & 1) * 2 * kBwdT;
+        v2[et] = l2;
+        v2[kBwdT + et] = dd;
+        mbar_arrive(BAR_VEC);
+      };
+      float l2n, ddn;
+      col_vals(0, l2n, ddn);
+      stage(step, l2n, ddn);
       bool stop = false;
-      for (int g = 0; g < p.G && !stop; ++g) {
-        const int h = kvh * p.G + g;
-        const int64_t rbase = (static_cast<int64_t>(b) * p.H + h) * p.N;
-        for (int t = kt; t <= t_hi; ++t, ++step) {
-          // stage lse2 and D of the tile's 128 query columns (two copies alternate;
-          // passing step s's barrier means every thread has finished step s - 1,
-          // so the copy written at step s + 1 is no longer read)
-          float *v2 = vec + (step & 1) * 2 * kBwdT;
-          const int qc = t * kBwdT + et;
-          v2[et] = qc < p.N ? p.lse[rbase + qc] * 1.4426950408889634f : INFINITY;
-          v2[kBwdT + et] = qc < p.N ? p.delta[rbase + qc] : 0.f;
-          mbar_arrive(BAR_VEC);
-          if (!mbar_wait(BAR_VEC, step & 1, abort_flag) ||
-              !mbar_wait(BAR_SF, s_cnt & 1, abort_flag) ||
-              !mbar_wait(BAR_DPF, s_cnt & 1, abort_flag)) {
-            stop = true;
-            break;
-          }
-          ++s_cnt;
-          tc_fence_after();
-          // allowed query columns of key row krow: i in [krow, krow + W - 1], i < N
-          const int c0 = t * kBwdT;
-          const bool full = kt * kBwdT + kBwdT - 1 <= c0 && c0 + kBwdT - 1 - kt * kBwdT <= p.W - 1 &&
-                            c0 + kBwdT <= p.N;
-          uint32_t mw[4];
-          col_mask(krow - c0, min(krow + p.W - 1, p.N - 1) - c0, mw);
-          const uint32_t tS = tmem + T_S + lane_off;
-          const uint32_t tP = tmem + T_DP + lane_off;
-#pragma unroll
-          for (int ch = 0; ch < kBwdT / 32; ++ch) {
-            uint32_t sr[32], dr[32];
-            tmem_ld32(tS + ch * 32, sr);
-            tmem_ld32(tP + ch * 32, dr);
-            uint32_t pk[16], dk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float pp[2], dd[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int c = 2 * i + e;
-                const int col = ch * 32 + c;
-                float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -v2[col]));
-                if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
-                pp[e] = pr;
-                dd[e] = pr * (__uint_as_float(dr[c]) - v2[kBwdT + col]);
-              }
-              pk[i] = pack_bf16(pp[0], pp[1]);
-              dk[i] = pack_bf16(dd[0], dd[1]);
-            }
-            tmem_st16_b(tS + ch * 16, pk);
-            tmem_st16_b(tP + ch * 16, dk);
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(BAR_EL);
+      for (int s = 0; s < n; ++s, ++step) {
+        const int t = kt + s % nqt;
+        if (s + 1 < n) col_vals(s + 1, l2n, ddn);  // loads in flight during this step
+        const float *v2 = vec + (step & 1) * 2 * kBwdT;
+        if (!mbar_wait(BAR_VEC, step & 1, abort_flag) ||
+            !mbar_wait(BAR_SF, s_cnt & 1, abort_flag)) {
+          stop = true;
+          break;
         }
+        tc_fence_after();
+        // allowed query columns of key row krow: i in [krow, krow + W - 1], i < N
+        const int c0 = t * kBwdT;
+        const bool full = kt * kBwdT + kBwdT - 1 <= c0 && c0 + kBwdT - 1 - kt * kBwdT <= p.W - 1 &&
+                          c0 + kBwdT <= p.N;
+        uint32_t mw[4];
+        col_mask(krow - c0, min(krow + p.W - 1, p.N - 1) - c0, mw);
+        const uint32_t tS = tmem + T_S + lane_off;
+        const uint32_t tP = tmem + T_DP + lane_off;
+        // phase 1: P^T (fp32 kept for dS), stored as bf16 over the low half of S^T
+        float pf[kBwdT];
+        auto pchunk = [&](int ch, const uint32_t (&sr)[32]) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 2 * i + e;
+              float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -v2[ch * 32 + c]));
+              if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
+              pf[ch * 32 + c] = pr;
+            }
+            pk[i] = pack_bf16(pf[ch * 32 + 2 * i], pf[ch * 32 + 2 * i + 1]);
+          }
+          tmem_st16_b(tS + ch * 16, pk);
+        };
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_issue(tS, r0);
+          tmem_ld32_issue(tS + 32, r1);
+          tmem_ld_wait2(r0, r1);
+          pchunk(0, r0);
+          tmem_ld32_issue(tS + 64, r0);
+          pchunk(1, r1);
+          tmem_ld32_issue(tS + 96, r1);
+          tmem_ld_wait2(r0, r1);
+          pchunk(2, r0);
+          pchunk(3, r1);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR_PF);
+        // phase 2: dS^T = P^T o (dP^T - D), stored as bf16 over the low half of dP^T
+        if (!mbar_wait(BAR_DPF, s_cnt & 1, abort_flag)) {
+          stop = true;
+          break;
+        }
+        ++s_cnt;
+        tc_fence_after();
+        auto dchunk = [&](int ch, const uint32_t (&dr)[32]) {
+          uint32_t dk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float dd[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 2 * i + e;
+              dd[e] = pf[ch * 32 + c] * (__uint_as_float(dr[c]) - v2[kBwdT + ch * 32 + c]);
+            }
+            dk[i] = pack_bf16(dd[0], dd[1]);
+          }
+          tmem_st16_b(tP + ch * 16, dk);
+        };
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_issue(tP, r0);
+          tmem_ld32_issue(tP + 32, r1);
+          tmem_ld_wait2(r0, r1);
+          dchunk(0, r0);
+          tmem_ld32_issue(tP + 64, r0);
+          dchunk(1, r1);
+          tmem_ld32_issue(tP + 96, r1);
+          tmem_ld_wait2(r0, r1);
+          dchunk(2, r0);
+          dchunk(3, r1);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR_DSF);
+        if (s + 1 < n) stage(step + 1, l2n, ddn);
       }
       if (stop || *abort_flag) break;
       if (!mbar_wait(BAR_AF, u_iter & 1, abort_flag)) break;
