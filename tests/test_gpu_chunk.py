@@ -77,6 +77,59 @@ def test_chunk_workload_sampled_rows(swa):
     ref = oracle.swa_chunk(q, kn, vn, rk, rv, qs, w.W, w.scale, rows=rows)
     got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_close(got, ref, what="chunk_ring workload")
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-2
+
+
+@pytest.mark.parametrize("needle_rel", [50, -1, 10])
+def test_chunk_needle_unaligned_ring(swa, needle_rel):
+    """A dominating key in the ring (past the wrap of an unaligned ring) or in the
+    chunk: query t sees it iff its position is in [q_start + t - W + 1, q_start + t]."""
+    W, Tq, d = 512, 256, 128
+    q_start = 4096 + 37
+    # needle_rel > 0 counts from the oldest ring position, < 0 from the newest,
+    # and 10 puts it in the chunk
+    p_star = q_start - W + needle_rel if needle_rel != 10 else q_start + 10
+    if needle_rel < 0:
+        p_star = q_start + needle_rel
+    u = np.zeros(d, dtype=np.float32)
+    u[:8] = 1.0
+    qf = np.tile(u, (1, 1, Tq, 1))
+    knf = si.bf16_bits_to_f32(si.normal_bf16(6, si.STREAM["k_new"], (1, 1, Tq, d))) * 0.1
+    rkf = si.bf16_bits_to_f32(si.normal_bf16(6, si.STREAM["k_ring"], (1, 1, W, d))) * 0.1
+    needle = 8.0 * u / np.linalg.norm(u) * math.sqrt(d)
+    if p_star >= q_start:
+        knf[0, 0, p_star - q_start] = needle
+    else:
+        rkf[0, 0, p_star % W] = needle  # slot = position mod W
+    q, kn, rk = (si.f32_to_bf16_bits(x.astype(np.float32)) for x in (qf, knf, rkf))
+    vn = si.normal_bf16(6, si.STREAM["v_new"], (1, 1, Tq, d))
+    rv = si.normal_bf16(6, si.STREAM["v_ring"], (1, 1, W, d))
+    scale = 1.0 / math.sqrt(d)
+    out, _, _, _ = _run(swa, q, kn, vn, rk, rv, [q_start], scale)
+    got = to_f64(out)[0, 0]
+    ref = oracle.swa_chunk(q, kn, vn, rk, rv, [q_start], W, scale)[0, 0]
+    assert_close(got, ref, what="chunk needle")
+    vsrc = vn[0, 0, p_star - q_start] if p_star >= q_start else rv[0, 0, p_star % W]
+    vneedle = si.bf16_bits_to_f32(vsrc).astype(np.float64)
+    for t in range(Tq):
+        sees = q_start + t - W + 1 <= p_star <= q_start + t
+        close = np.max(np.abs(got[t] - vneedle)) < 0.05
+        assert close == sees, f"query {t}: sees needle {sees}, output matches {close}"
+
+
+def test_chunk_shift_by_window_is_identical(swa):
+    """The same ring contents at q_start and q_start + W hold the same relative
+    positions (slot = position mod W), so the outputs are bit-identical."""
+    B, H, Hkv, Tq, d, W = 2, 8, 2, 200, 128, 384
+    starts = [5000 + 77, 1000]
+    seed = 55
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    a, la, _, _ = _run(swa, q, kn, vn, rk, rv, starts, 0.1)
+    b, lb, _, _ = _run(swa, q, kn, vn, rk, rv, [s + W for s in starts], 0.1)
+    assert torch.equal(a, b) and torch.equal(la, lb)
 
 
 def test_chunked_equals_full_prefill(swa):

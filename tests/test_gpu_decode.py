@@ -127,3 +127,15 @@ def test_decode_sink_workload_all_rows(swa):
     assert swa.swa_get_device_status() == 0
     ref = oracle.swa_decode_sink(q, rk, rv, sk, sv, pos, w.W, w.scale)
     assert_close_bf16out(to_f64(out), ref, what="decode sink workload")
+
+
+def test_decode_shift_by_window_is_identical(swa):
+    """pos and pos + W see the same slots at the same relative positions."""
+    B, H, Hkv, d, W = 4, 16, 4, 128, 1024
+    pos = [5000, 1023, 77777, 2048]
+    q = si.normal_bf16(61, si.STREAM["q"], (B, H, d))
+    rk = si.normal_bf16(61, si.STREAM["k_ring"], (B, Hkv, W, d))
+    rv = si.normal_bf16(61, si.STREAM["v_ring"], (B, Hkv, W, d))
+    a, la = _run(swa, q, rk, rv, pos, 0.09)
+    b, lb = _run(swa, q, rk, rv, [p + W for p in pos], 0.09)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)

@@ -90,6 +90,9 @@ def test_workload_sampled_rows(swa, name):
     ref = oracle.swa_forward(q, k, v, w.W, w.scale, rows=rows)
     got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_close(got, ref, what=name)
+    # relative RMS error: outputs here are ~0.02 in size, so also bound the error
+    # relative to them (bf16 rounding of the output alone is ~2^-9 relative)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-2
 
 
 @pytest.mark.parametrize("W,needle", [(64, 100), (64, 127), (64, 128), (512, 511), (512, 512),
