@@ -35,6 +35,28 @@ def test_header_declares_the_boundary():
         assert want in names
 
 
+def test_header_is_plain_c(tmp_path):
+    """The boundary header compiles as strict C99 and links against the library:
+    plain pointers and sizes, no C++ or torch types."""
+    import shutil
+    import subprocess
+
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "swa.h"\n'
+                   "int main(void) { return swa_version() > 0 && "
+                   "swa_status_string(0) != 0 ? 0 : 1; }\n")
+    from sliding_window_sparse_b200 import build
+
+    lib = build.build()
+    exe = tmp_path / "use_header"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), str(lib),
+                    "-Wl,-rpath," + os.path.dirname(str(lib))], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
 def test_every_declared_symbol_is_exported(native):
     lib = native.lib()
     for name in declared_symbols():
