@@ -27,6 +27,7 @@ Functions and the passages they follow (page title, section):
 * :func:`swa_varlen`      -- blog section 5.2 tip 4 (packed batches, windows per
                              sequence via cu_seqlens), with optional sinks.
 * :func:`swa_decode_sink` -- taxonomy page section 3.2 on top of the ring decode.
+* :func:`swa_chunk_sink`  -- taxonomy page section 3.2 on top of the chunked prefill.
 * :func:`swa_backward`    -- M003 note sections 07-08 (Q/K/V gradients under the
                              same mask); :func:`swa_forward_f64` is the forward
                              on fp64 inputs that its finite differences use.
@@ -106,6 +107,9 @@ def _configure(lib):
     lib.orc_swa_decode_sink.restype = _i64
     lib.orc_swa_decode_sink.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int,
                                         _int, _i64, _i64, _dbl, _ptr, _ptr]
+    lib.orc_swa_chunk_sink.restype = _i64
+    lib.orc_swa_chunk_sink.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _ptr, _int,
+                                       _int, _int, _i64, _int, _i64, _dbl, _ptr, _i64, _ptr, _ptr]
     lib.orc_swa_forward_f64.restype = _i64
     lib.orc_swa_forward_f64.argtypes = [_ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
                                         _dbl, _ptr]
@@ -297,6 +301,30 @@ def swa_chunk(q, k_new, v_new, ring_k, ring_v, q_start, W: int, scale: float, ro
     lse = np.empty(n, dtype=np.float64) if with_lse else None
     bad = _load().orc_swa_chunk(_p(q), _p(k_new), _p(v_new), _p(ring_k), _p(ring_v), _p(qs),
                                 B, H, Hkv, Tq, d, W, scale, _p(r), n, _p(out), _p(lse))
+    if bad:
+        raise ValueError(f"{bad} query rows have a missing or no legal key")
+    if r is None:
+        out = out.reshape(B, H, Tq, d)
+        if lse is not None:
+            lse = lse.reshape(B, H, Tq)
+    return (out, lse) if with_lse else out
+
+
+def swa_chunk_sink(q, k_new, v_new, ring_k, ring_v, sink_k, sink_v, q_start, W: int,
+                   scale: float, rows=None, with_lse=False):
+    """swa_chunk with sink rows [B,Hkv,S,d] holding positions 0..S-1."""
+    q, k_new, v_new = _u16(q), _u16(k_new), _u16(v_new)
+    ring_k, ring_v, sink_k, sink_v = _u16(ring_k), _u16(ring_v), _u16(sink_k), _u16(sink_v)
+    B, H, Tq, d = q.shape
+    Hkv, S = k_new.shape[1], sink_k.shape[2]
+    qs = np.ascontiguousarray(q_start, dtype=np.int64).reshape(B)
+    r = _rows(rows)
+    n = r.shape[0] if r is not None else B * H * Tq
+    out = np.empty((n, d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64) if with_lse else None
+    bad = _load().orc_swa_chunk_sink(_p(q), _p(k_new), _p(v_new), _p(ring_k), _p(ring_v),
+                                     _p(sink_k), _p(sink_v), S, _p(qs), B, H, Hkv, Tq, d, W,
+                                     scale, _p(r), n, _p(out), _p(lse))
     if bad:
         raise ValueError(f"{bad} query rows have a missing or no legal key")
     if r is None:

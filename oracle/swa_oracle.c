@@ -645,6 +645,69 @@ int64_t orc_swa_forward_f64(const double *q, const double *k, const double *v, i
 }
 
 /*
+ * Chunked prefill over a ring cache with attention sinks ([CH10 s10.2] with
+ * [TAXO s3.2]).  As orc_swa_chunk, and in addition sink_k, sink_v:
+ * [B, Hkv, S, d] hold positions 0 .. S-1 (written once, never evicted).
+ * Query t at position p = q_start[b] + t reads every position j with
+ * allowed_sink(p, j, W, S) in increasing order: from the chunk if
+ * j >= q_start[b], from the ring if it is one of the last W positions before
+ * the chunk and inside the window, else (a sink before the window) from the
+ * sink rows.  Returns the number of rows with a missing or no legal key.
+ */
+int64_t orc_swa_chunk_sink(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                           const uint16_t *ring_k, const uint16_t *ring_v,
+                           const uint16_t *sink_k, const uint16_t *sink_v, int64_t S,
+                           const int64_t *q_start, int B, int H, int Hkv, int64_t Tq, int d,
+                           int64_t W, double scale, const int64_t *rows, int64_t n_rows,
+                           double *out, double *lse)
+{
+    int64_t total = rows ? n_rows : (int64_t)B * H * Tq;
+    int64_t bad = 0;
+    int64_t *maps = (int64_t *)malloc(sizeof(int64_t) * (size_t)(B * W));
+    for (int64_t b = 0; b < B; ++b) orc_ring_positions(q_start[b], W, maps + b * W);
+#pragma omp parallel reduction(+ : bad)
+    {
+        int64_t cap = W + Tq + S;
+        const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)cap);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)cap);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < total; ++r) {
+            int64_t b, h, t;
+            row_of(rows, r, H, Tq, &b, &h, &t);
+            int64_t kh = kv_head(h, H, Hkv);
+            int64_t p = q_start[b] + t;
+            int64_t n = 0, missing = 0;
+            for (int64_t j = 0; j <= p; ++j) {
+                if (!allowed_sink(p, j, W, S)) continue;
+                if (j >= q_start[b]) {
+                    int64_t row = j - q_start[b];
+                    kr[n] = k_new + ((b * Hkv + kh) * Tq + row) * d;
+                    vr[n] = v_new + ((b * Hkv + kh) * Tq + row) * d;
+                } else if (j >= p - W + 1) {
+                    int64_t s = find_slot(maps + b * W, W, j);
+                    if (s < 0) { ++missing; continue; }
+                    kr[n] = ring_k + ((b * Hkv + kh) * W + s) * d;
+                    vr[n] = ring_v + ((b * Hkv + kh) * W + s) * d;
+                } else {
+                    kr[n] = sink_k + ((b * Hkv + kh) * S + j) * d;
+                    vr[n] = sink_v + ((b * Hkv + kh) * S + j) * d;
+                }
+                ++n;
+            }
+            const uint16_t *qrow = q + ((b * H + h) * Tq + t) * d;
+            int e = attend_one(qrow, kr, vr, n, d, scale, out + r * d, lse ? lse + r : NULL, sc);
+            if (e || missing) ++bad;
+        }
+        free(kr);
+        free(vr);
+        free(sc);
+    }
+    free(maps);
+    return bad;
+}
+
+/*
  * Tile classification by brute force ([M003 s04]): every in-range
  * (query, key) coordinate of a tile is tested with the visibility rule; a tile
  * whose in-range pairs are all forbidden is skipped (class 0), one whose

@@ -92,6 +92,8 @@ def _pin_suite(golden_dir):
         lambda: pins.test_sink_tokens_influence_and_middle_tokens_do_not(),
         lambda: pins.test_decode_sink_equals_prefill_row(8, 4, 12),
         lambda: pins.test_decode_sink_equals_prefill_row(16, 4, 50),
+        lambda: pins.test_chunked_with_sinks_equals_full(16, 4, [(0, 5), (5, 40), (40, 41),
+                                                                  (41, 90)]),
         lambda: pins.test_forward_f64_equals_forward(),
         lambda: pins.test_backward_finite_differences(3),
         lambda: pins.test_backward_full_window_equals_torch_autograd(1, 4, 2, 37, 16),

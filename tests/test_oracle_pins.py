@@ -549,6 +549,36 @@ def test_decode_sink_equals_prefill_row(W, S, P):
         assert np.array_equal(dec, plain)
 
 
+@pytest.mark.parametrize("W,S,chunks", [(16, 4, [(0, 5), (5, 40), (40, 41), (41, 90)]),
+                                         (8, 2, [(0, 30), (30, 31), (31, 70)]),
+                                         (32, 4, [(0, 2), (2, 100)])])
+def test_chunked_with_sinks_equals_full(W, S, chunks):
+    """Chunks over a ring plus sink rows reproduce the one-pass prefill with the
+    same sinks exactly (taxonomy page section 3.2 on Chapter 10 section 10.2)."""
+    B, H, Hkv, d = 2, 4, 2, 8
+    N = chunks[-1][1]
+    q = _rand(35, (B, H, N, d), si.STREAM["q"])
+    k = _rand(35, (B, Hkv, N, d), si.STREAM["k"])
+    v = _rand(35, (B, Hkv, N, d), si.STREAM["v"])
+    full = []
+    for b in range(B):
+        tm = lambda x: np.ascontiguousarray(x[b].transpose(1, 0, 2))
+        full.append(oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, 0.45, n_sink=S)
+                    .transpose(1, 0, 2))
+    sk = np.ascontiguousarray(k[:, :, :S])
+    sv = np.ascontiguousarray(v[:, :, :S])
+    rk = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rv = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    for a, e in chunks:
+        sl = (slice(None), slice(None), slice(a, e))
+        out = oracle.swa_chunk_sink(np.ascontiguousarray(q[sl]), np.ascontiguousarray(k[sl]),
+                                    np.ascontiguousarray(v[sl]), rk, rv, sk, sv, [a] * B, W, 0.45)
+        for b in range(B):
+            assert np.array_equal(out[b], full[b][:, a:e])
+        rk, rv = oracle.ring_update(np.ascontiguousarray(k[sl]), np.ascontiguousarray(v[sl]),
+                                    rk, rv, [a] * B, W)
+
+
 # --- gradients (M003 note section 07: finite-difference check of Q/K/V gradients) ----
 
 def _f64_inputs(seed, B, H, Hkv, N, d):
