@@ -84,7 +84,9 @@ def useful_flops(w) -> int:
 
         return 4 * w.d * w.H * sum(sequence_pairs(int(n), w.W, w.n_sink) for n in seq_lens(w))
     if w.kind == "chunk":
-        pairs = sum(valid_pairs_row(w.q_start + t, w.W) for n in chunk_rows(w) for t in range(n))
+        pairs = sum(valid_pairs_row(w.q_start + t, w.W) +
+                    min(w.n_sink, max(0, w.q_start + t - w.W + 1))
+                    for n in chunk_rows(w) for t in range(n))
         return 4 * w.d * w.H * pairs
     raise ValueError(w.kind)
 
@@ -159,7 +161,7 @@ def describe(w) -> str:
     if w.kind == "chunk":
         rows = f" valid rows U[{w.len_lo},{w.len_hi}]" if w.len_hi else ""
         return (f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} Tq{w.Tq} d{w.d} W{w.W} "
-                f"q_start{w.q_start}{rows}")
+                f"q_start{w.q_start}{rows}{sink}")
     return (f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} d{w.d} W{w.W} "
             f"ctx U[{w.ctx_lo},{w.ctx_hi}]{sink}")
 
@@ -299,6 +301,9 @@ def make_inputs(w, device, seed_offset=0):
              "q_start": torch.full((w.B,), w.q_start, dtype=torch.int64, device=device)}
         if w.len_hi:
             x["chunk_len"] = torch.tensor(chunk_rows(w), dtype=torch.int64, device=device)
+        if w.n_sink:
+            x["k_sink"] = g("k_sink", (w.B, w.Hkv, w.n_sink, w.d))
+            x["v_sink"] = g("v_sink", (w.B, w.Hkv, w.n_sink, w.d))
         return x
     from swa_inputs import uniform_int
 
@@ -340,7 +345,8 @@ def make_call(w, x, swa):
                 x["q"], x["k_new"], x["v_new"], x["k_ring"], x["v_ring"], x["q_start"],
                 x["chunk_len"], w.scale, out=out), out, 1)
         return (lambda: swa.swa_attn_chunk_ring(x["q"], x["k_new"], x["v_new"], x["k_ring"],
-                                                x["v_ring"], x["q_start"], w.scale, out=out),
+                                                x["v_ring"], x["q_start"], w.scale, out=out,
+                                                k_sink=x.get("k_sink"), v_sink=x.get("v_sink")),
                 out, 1)
     out = torch.empty_like(x["q"])
     ws = torch.empty(swa.swa_decode_workspace_bytes(w.B, w.H, w.Hkv, w.d, w.W), dtype=torch.uint8,
@@ -547,7 +553,7 @@ def run_native(args):
     if not args.headline_only:
         for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring",
                      "varlen_prefill", "mistral_prefill_sink", "chunk_ring_ragged",
-                     "decode_ring_sink", "mistral_backward"):
+                     "decode_ring_sink", "chunk_ring_sink", "mistral_backward"):
             if name == headline:
                 continue
             pw = WORKLOADS[name]

@@ -204,6 +204,27 @@ SWA_API int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_
                         int update_ring, void *stream);
 
 /*
+ * swa_attn_chunk_ring_sink -- swa_attn_chunk_ring with attention sinks.
+ * Passage: sparse-attention taxonomy page section 3.2 (StreamingLLM keeps the
+ * first tokens visible besides the recent W) over Chapter 10 section 10.2.
+ * Query t at position p = q_start[b] + t reads key j iff j <= p and
+ * (j >= p - W + 1 or j < n_sink): positions in the window from the ring and
+ * the chunk as in swa_attn_chunk_ring, the sinks before the window from
+ * k_sink / v_sink.
+ *   k_sink, v_sink: [B, Hkv, n_sink, d] bf16, device: row j holds position j
+ *      for every j < n_sink, written by the caller before the call (for a
+ *      chunk that contains some of them, copy those rows from k_new / v_new
+ *      first).  1 <= n_sink <= 128.  The ring update leaves them untouched.
+ * Other arguments, layouts and limits as swa_attn_chunk_ring.
+ */
+SWA_API int swa_attn_chunk_ring_sink(const void *q, const void *k_new, const void *v_new,
+                                     void *k_ring, void *v_ring, const void *k_sink,
+                                     const void *v_sink, int n_sink, const int64_t *q_start,
+                                     void *out, float *lse, int B, int H, int Hkv, int64_t Tq,
+                                     int d, int64_t W, float scale, int update_ring,
+                                     void *stream);
+
+/*
  * swa_attn_chunk_ring_ragged -- swa_attn_chunk_ring for a batch whose chunks
  * have different lengths (Chapter 10 section 10.2 applied per sequence; the
  * window is per sequence, as the blog's troubleshooting section 5.2 stresses

@@ -30,6 +30,7 @@ __all__ = [
     "swa_attn_varlen",
     "swa_attn_chunk_ring",
     "swa_attn_chunk_ring_ragged",
+    "swa_attn_chunk_ring_sink",
     "swa_ring_write",
     "swa_decode_workspace_bytes",
     "swa_attn_decode_ring",
@@ -187,8 +188,13 @@ def swa_attn_varlen(q, k, v, cu_seqlens, max_seqlen: int, W: int, scale: float |
 
 
 def swa_attn_chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, scale: float | None = None,
-                        update_ring: bool = False, out=None, lse=None, return_lse: bool = False):
-    """Chunked prefill on a ring cache: q [B,H,Tq,d], chunk k/v [B,Hkv,Tq,d], ring [B,Hkv,W,d]."""
+                        update_ring: bool = False, out=None, lse=None, return_lse: bool = False,
+                        k_sink=None, v_sink=None):
+    """Chunked prefill on a ring cache: q [B,H,Tq,d], chunk k/v [B,Hkv,Tq,d], ring [B,Hkv,W,d].
+
+    With k_sink / v_sink [B,Hkv,S,d] (positions 0..S-1) the sinks before each window
+    are attended too (swa_attn_chunk_ring_sink).
+    """
     for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"),
                  (v_ring, "v_ring")):
         _need(t, n, dims=4)
@@ -201,10 +207,21 @@ def swa_attn_chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, scale: float |
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
-    check("swa_attn_chunk_ring",
-          lib().swa_attn_chunk_ring(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring),
-                                    _ptr(q_start), _ptr(out), _ptr(lse), B, H, Hkv, Tq, d, W,
-                                    scale, 1 if update_ring else 0, _stream(q.device)))
+    if k_sink is not None:
+        _need(k_sink, "k_sink", dims=4)
+        _need(v_sink, "v_sink", dims=4)
+        check("swa_attn_chunk_ring_sink",
+              lib().swa_attn_chunk_ring_sink(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring),
+                                             _ptr(v_ring), _ptr(k_sink), _ptr(v_sink),
+                                             k_sink.shape[2], _ptr(q_start), _ptr(out), _ptr(lse),
+                                             B, H, Hkv, Tq, d, W, scale, 1 if update_ring else 0,
+                                             _stream(q.device)))
+    else:
+        check("swa_attn_chunk_ring",
+              lib().swa_attn_chunk_ring(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring),
+                                        _ptr(v_ring), _ptr(q_start), _ptr(out), _ptr(lse), B, H,
+                                        Hkv, Tq, d, W, scale, 1 if update_ring else 0,
+                                        _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

@@ -71,7 +71,8 @@ struct Fwd2Params {
   int n_q = 0;             // query rows per (b, h); MODE 2: longest sequence
   int n_k = 0;             // rows of the main key source (N, or Tq for a chunk)
   int64_t W = 0;           // window (MODE 0 / 2: clamped to n_q + kQT)
-  int n_sink = 0;          // MODE 0 / 2: keys 0 .. n_sink-1 stay visible to later queries
+  int n_sink = 0;          // keys 0 .. n_sink-1 stay visible to later queries (MODE 1: from
+                           // their own rows, the tensor maps tm_ks / tm_vs)
   float scale_log2 = 0.f;  // scale * log2(e)
   int nqt = 0;             // query tiles per (b, h)
   int n_ring_tiles = 0;    // MODE 1: ceil(W / kKT)
@@ -152,15 +153,17 @@ struct Walker2 {
   bool full_ring;
   bool has_b;
   int live_a_end, live_b_begin;  // MODE 0: A is live on [kt, live_a_end], B on [live_b_begin, kt_end)
-  int n_sink;        // MODE 0 / 2: sink keys 0 .. n_sink-1
-  bool sink_pending;  // tile 0 (sinks only) still to be yielded ahead of kt
+  int n_sink;        // sink keys 0 .. n_sink-1
+  bool sink_pending;  // the sink tile (MODE 0 / 2: key tile 0; MODE 1: the sink rows, k = -1)
+                      // still to be yielded ahead of kt
+  int sink_vis[2];    // MODE 1: sinks before the window of the tile's last row
 
   // len: valid query rows of this unit's sequence (MODE 1: also its chunk keys)
   __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs, int len) {
     has_b = U.has_b;
     n_k = MODE == 0 ? p.n_k : len;
     W = static_cast<int>(p.W);
-    n_sink = (SINK && MODE != 1) ? p.n_sink : 0;
+    n_sink = SINK ? p.n_sink : 0;
     sink_pending = false;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
@@ -184,6 +187,15 @@ struct Walker2 {
       kt_end = nrt + (len + kKT - 1) / kKT;
       full_ring = qs >= p.W;
       wrap = static_cast<int>(full_ring ? qs % p.W : qs);
+      if (SINK) {
+        // query row r sees sink j iff j < n_sink and j < qs + r - W + 1
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int64_t v = qs + qhi[x] - p.W + 1;
+          sink_vis[x] = static_cast<int>(v < 0 ? 0 : (v > n_sink ? n_sink : v));
+        }
+        sink_pending = n_sink > 0 && (sink_vis[0] > 0 || (has_b && sink_vis[1] > 0));
+      }
     }
   }
 
@@ -267,6 +279,15 @@ struct Walker2 {
   // Tile 0 under sinks is partial unless the window alone covers it.
   __device__ __forceinline__ bool next(int &k, int &src, int &y0, int &ca, int &cb) {
     int lo[2], hi[2], base[2];
+    if (SINK && MODE == 1 && sink_pending) {
+      sink_pending = false;
+      k = -1;
+      src = 2;
+      y0 = 0;
+      ca = sink_vis[0] > 0 ? 2 : 0;
+      cb = (has_b && sink_vis[1] > 0) ? 2 : 0;
+      return true;
+    }
     if (SINK && MODE != 1 && sink_pending) {
       sink_pending = false;
       k = 0;
@@ -294,7 +315,9 @@ template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kFwd2Threads, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_vr, const Fwd2Params p) {
+                const __grid_constant__ CUtensorMap tm_vr,
+                const __grid_constant__ CUtensorMap tm_ks,
+                const __grid_constant__ CUtensorMap tm_vs, const Fwd2Params p) {
   using L = Fwd2Layout<D>;
   constexpr int NK = L::NK, NV = L::NV;
   extern __shared__ uint8_t smem_raw[];
@@ -345,6 +368,10 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     if (MODE == 1) {
       tma_prefetch_desc(&tm_kr);
       tma_prefetch_desc(&tm_vr);
+    }
+    if (MODE == 1 && SINK) {
+      tma_prefetch_desc(&tm_ks);
+      tma_prefetch_desc(&tm_vs);
     }
   }
   tc_fence_before();
@@ -424,8 +451,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         const int z = MODE == 2 ? static_cast<int>(qs) : U.b * p.Hkv + U.kvh;
         while (wk.next_live(k, src, y0, ca, cb)) {
           const int sk = kv_iter % NK, sv = kv_iter % NV;
-          const CUtensorMap *mk = src == 1 ? &tm_kr : &tm_k;
-          const CUtensorMap *mv = src == 1 ? &tm_vr : &tm_v;
+          const CUtensorMap *mk = src == 1 ? &tm_kr : (src == 2 ? &tm_ks : &tm_k);
+          const CUtensorMap *mv = src == 1 ? &tm_vr : (src == 2 ? &tm_vs : &tm_v);
           if (kv_iter >= NK && !mbar_wait(BAR_KE + 8 * sk, ((kv_iter / NK) - 1) & 1, abort_flag))
             break;
           mbar_expect_tx(BAR_KF + 8 * sk, L::KV_BYTES);
@@ -596,15 +623,22 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         if (cls == 2) {
           // allowed columns of this row: c in a segment with base + c in [q - W + 1, q],
           // as a 128-bit mask (one word per 32 columns)
-          int lo[2], hi[2], base[2], s_, y_;
-          wk.segments(k, lo, hi, base, s_, y_);
+          int lo[2] = {1, 1}, hi[2] = {0, 0}, base[2], s_, y_;
+          int sink_hi = -1;
+          if (SINK && MODE == 1 && k < 0) {
+            // the sink rows: columns below min(n_sink, q - W + 1) (q absolute)
+            const int64_t v = qs + qrow - wk.W + 1;
+            sink_hi = static_cast<int>(v < 0 ? 0 : (v > wk.n_sink ? wk.n_sink : v)) - 1;
+          } else {
+            wk.segments(k, lo, hi, base, s_, y_);
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            lo[g] = max(lo[g], qrow - wk.W + 1 - base[g]);
-            hi[g] = min(hi[g], qrow - base[g]);
+            for (int g = 0; g < 2; ++g) {
+              lo[g] = max(lo[g], qrow - wk.W + 1 - base[g]);
+              hi[g] = min(hi[g], qrow - base[g]);
+            }
+            // sinks: columns 0 .. n_sink-1 of tile 0, up to the row itself
+            if (SINK && MODE != 1 && k == 0) sink_hi = min(wk.n_sink - 1, qrow);
           }
-          // sinks: columns 0 .. n_sink-1 of tile 0, up to the row itself
-          const int sink_hi = (SINK && MODE != 1 && k == 0) ? min(wk.n_sink - 1, qrow) : -1;
           uint32_t mw[kKT / 32];
 #pragma unroll
           for (int w = 0; w < kKT / 32; ++w)

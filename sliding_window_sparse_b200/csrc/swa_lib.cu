@@ -98,10 +98,12 @@ int common_checks(int B, int H, int Hkv, int d, int64_t W, float scale) {
   return SWA_OK;
 }
 
+// tks / tvs: the sink rows of the chunk-ring path with sinks (any map otherwise)
 template <int D, int MODE, bool SINK = false>
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                const CUtensorMap &tkr, const CUtensorMap &tvr, swa::Fwd2Params p,
-               cudaStream_t st) {
+               cudaStream_t st, const CUtensorMap *tks = nullptr,
+               const CUtensorMap *tvs = nullptr) {
   using L = swa::Fwd2Layout<D>;
   auto kern = swa::fwd2_kernel<D, MODE, SINK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
@@ -118,7 +120,8 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
     return SWA_ERR_CUDA;
   const int grid = static_cast<int>(units < sms ? units : sms);
-  kern<<<grid, swa::kFwd2Threads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr, p);
+  kern<<<grid, swa::kFwd2Threads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr, tks ? *tks : tk,
+                                                   tvs ? *tvs : tv, p);
   return check_launch();
 }
 
@@ -332,7 +335,8 @@ namespace {
 int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring, void *v_ring,
                const int64_t *q_start, const int64_t *chunk_len, void *out, float *lse, int B,
                int H, int Hkv, int64_t Tq, int d, int64_t W, float scale, int update_ring,
-               void *stream) {
+               void *stream, const void *k_sink = nullptr, const void *v_sink = nullptr,
+               int n_sink = 0) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k_new || !v_new || !k_ring || !v_ring || !q_start || !out) return SWA_ERR_INVALID_ARG;
@@ -340,12 +344,20 @@ int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring
       !aligned16(v_ring) || !aligned16(out))
     return SWA_ERR_INVALID_ARG;
   if (Tq < 1 || Tq >= (int64_t(1) << 29) || W >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
-  CUtensorMap tq, tk, tv, tkr, tvr;
+  if (n_sink < 0 || n_sink > kBK) return SWA_ERR_INVALID_ARG;
+  if (n_sink > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink)))
+    return SWA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tkr, tvr, tks, tvs;
   if ((e = make_map(&tq, q, d, Tq, static_cast<int64_t>(B) * H, kBQ))) return e;
   if ((e = make_map(&tk, k_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tv, v_new, d, Tq, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tkr, k_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
   if ((e = make_map(&tvr, v_ring, d, W, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  if (n_sink > 0) {
+    // one 128-row box over the n_sink rows: the rows past them read as zero
+    if ((e = make_map(&tks, k_sink, d, n_sink, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+    if ((e = make_map(&tvs, v_sink, d, n_sink, static_cast<int64_t>(B) * Hkv, kBK))) return e;
+  }
   swa::Fwd2Params p;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.lse = lse;
@@ -358,12 +370,17 @@ int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring
   p.n_q = static_cast<int>(Tq);
   p.n_k = static_cast<int>(Tq);
   p.W = W;
+  p.n_sink = n_sink;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.nqt = static_cast<int>((Tq + kBQ - 1) / kBQ);
   p.n_ring_tiles = static_cast<int>((W + kBK - 1) / kBK);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = d == 128 ? launch_fwd<128, 1>(tq, tk, tv, tkr, tvr, p, st)
-               : launch_fwd<64, 1>(tq, tk, tv, tkr, tvr, p, st);
+  if (n_sink > 0)
+    e = d == 128 ? launch_fwd<128, 1, true>(tq, tk, tv, tkr, tvr, p, st, &tks, &tvs)
+                 : launch_fwd<64, 1, true>(tq, tk, tv, tkr, tvr, p, st, &tks, &tvs);
+  else
+    e = d == 128 ? launch_fwd<128, 1>(tq, tk, tv, tkr, tvr, p, st)
+                 : launch_fwd<64, 1>(tq, tk, tv, tkr, tvr, p, st);
   if (e || !update_ring) return e;
   return ring_write(k_new, v_new, k_ring, v_ring, q_start, chunk_len, B, Hkv, Tq, d, W, stream);
 }
@@ -375,6 +392,16 @@ int swa_attn_chunk_ring(const void *q, const void *k_new, const void *v_new, voi
                         int update_ring, void *stream) {
   return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, nullptr, out, lse, B, H, Hkv, Tq, d,
                     W, scale, update_ring, stream);
+}
+
+int swa_attn_chunk_ring_sink(const void *q, const void *k_new, const void *v_new,
+                             void *k_ring, void *v_ring, const void *k_sink, const void *v_sink,
+                             int n_sink, const int64_t *q_start, void *out, float *lse, int B,
+                             int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                             int update_ring, void *stream) {
+  if (n_sink < 1) return SWA_ERR_INVALID_ARG;
+  return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, nullptr, out, lse, B, H, Hkv, Tq, d,
+                    W, scale, update_ring, stream, k_sink, v_sink, n_sink);
 }
 
 int swa_attn_chunk_ring_ragged(const void *q, const void *k_new, const void *v_new,

@@ -67,6 +67,9 @@ WORKLOADS = {
     "decode_ring_sink": Workload("decode_ring_sink", "decode", B=64, H=32, Hkv=8, d=128, W=4096,
                                  ctx_lo=4096, ctx_hi=131072, n_sink=4, seed=8,
                                  note="batched decode with 4 attention sinks"),
+    "chunk_ring_sink": Workload("chunk_ring_sink", "chunk", B=4, H=32, Hkv=8, d=128, W=4096,
+                                Tq=512, q_start=12288, n_sink=4, seed=10,
+                                note="chunked prefill on a ring cache with 4 attention sinks"),
     "mistral_backward": Workload("mistral_backward", "backward", B=1, H=32, Hkv=8, d=128, W=4096,
                                  N=8192, seed=9, note="gradients of the Mistral-shaped prefill"),
 }
@@ -100,7 +103,7 @@ def varlen_inputs(w: Workload):
 
 
 def sink_inputs(w: Workload):
-    """Sink rows [B, Hkv, n_sink, d] of a decode workload."""
+    """Sink rows [B, Hkv, n_sink, d] of a decode or chunk workload."""
     k = normal_bf16(w.seed, STREAM["k_sink"], (w.B, w.Hkv, w.n_sink, w.d))
     v = normal_bf16(w.seed, STREAM["v_sink"], (w.B, w.Hkv, w.n_sink, w.d))
     return k, v

@@ -266,3 +266,56 @@ def test_ragged_chunk_workload_sampled_rows(swa):
                                w.W, w.scale, rows=rows)
         assert_close(got[b, rows[:, 1], rows[:, 2]], ref, what=f"ragged chunk workload b={b}")
         assert np.all(got[b, :, n:] == 7.0)
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,d,W,S,starts", [
+    (2, 8, 2, 200, 128, 256, 4, [5000 + 77, 300]),   # head pairs, sinks before the window
+    (3, 6, 2, 130, 64, 100, 16, [1000, 77, 3]),      # query-tile pairs; a start below S
+    (1, 4, 2, 64, 128, 512, 4, [10]),                # no query sees a sink: sink tile skipped
+    (1, 2, 1, 300, 128, 128, 128, [4096]),           # a full tile of sinks
+])
+def test_chunk_with_sinks(swa, B, H, Hkv, Tq, d, W, S, starts):
+    """Chunk over the ring plus sink rows (taxonomy page section 3.2) vs the oracle."""
+    from tests._util import assert_close_bf16out
+
+    seed = 1200 + Tq + W + S
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    sk = si.normal_bf16(seed, si.STREAM["k_sink"], (B, Hkv, S, d))
+    sv = si.normal_bf16(seed, si.STREAM["v_sink"], (B, Hkv, S, d))
+    for b, qs in enumerate(starts):  # sink positions inside the chunk: its own rows
+        for j in range(qs, min(S, qs + Tq)):
+            sk[b, :, j] = kn[b, :, j - qs]
+            sv[b, :, j] = vn[b, :, j - qs]
+    scale = 1.0 / math.sqrt(d)
+    tq, tkn, tvn, trk, trv = (to_dev(x) for x in (q, kn, vn, rk, rv))
+    out, lse = swa.swa_attn_chunk_ring(tq, tkn, tvn, trk, trv,
+                                       torch.tensor(starts, dtype=torch.int64, device="cuda"),
+                                       scale, return_lse=True, k_sink=to_dev(sk),
+                                       v_sink=to_dev(sv))
+    assert swa.swa_get_device_status() == 0
+    ref, ref_lse = oracle.swa_chunk_sink(q, kn, vn, rk, rv, sk, sv, starts, W, scale,
+                                         with_lse=True)
+    assert_close_bf16out(to_f64(out), ref, what="chunk with sinks")
+    assert np.max(np.abs(to_f64(lse) - ref_lse)) < 1e-3
+
+
+def test_chunk_sink_workload_sampled_rows(swa):
+    """The benchmarked chunk-ring workload with 4 sinks, sampled rows."""
+    from swa_inputs.workloads import sink_inputs
+    from tests._util import assert_close_bf16out
+
+    w = WORKLOADS["chunk_ring_sink"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    sk, sv = sink_inputs(w)
+    out = swa.swa_attn_chunk_ring(to_dev(q), to_dev(kn), to_dev(vn), to_dev(rk), to_dev(rv),
+                                  torch.tensor(qs, dtype=torch.int64, device="cuda"), w.scale,
+                                  k_sink=to_dev(sk), v_sink=to_dev(sv))
+    assert swa.swa_get_device_status() == 0
+    edges = [0, 1, 127, 128, 255, 256, 383, 384, 510, 511]
+    rows = sample_rows(w.B, w.H, w.Tq, 200, seed=13, extra=edges)
+    ref = oracle.swa_chunk_sink(q, kn, vn, rk, rv, sk, sv, qs, w.W, w.scale, rows=rows)
+    got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert_close_bf16out(got, ref, what="chunk_ring_sink workload")
