@@ -55,7 +55,9 @@ def assert_close_bf16out(got, ref, what=""):
     plus sinks) can have |o| of 2 to 4, where half an ulp of bf16 is already
     3.9e-3 to 7.8e-3; the bf16 weights P add at most 2^-8 * max|v| more.  The
     bound |err| <= MAX_ABS + 2^-8 * |ref| keeps MAX_ABS for the weights and
-    rounds the output on top; mean-abs stays at MEAN_ABS.
+    rounds the output on top.  Rounding errors average to about half of their
+    bound, so mean-abs <= MEAN_ABS + 2^-9 * mean|ref|; both extra terms vanish
+    for the many-key rows of the benchmark workloads, whose |o| is ~0.02.
     """
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
@@ -63,8 +65,10 @@ def assert_close_bf16out(got, ref, what=""):
     diff = np.abs(got - ref)
     excess = diff - (MAX_ABS + BF16_U * np.abs(ref))
     mx, mn = float(diff.max()), float(diff.mean())
-    assert excess.max() <= 0 and mn <= MEAN_ABS, \
-        f"{what}: max-abs {mx:.3e} (over the bound by {excess.max():.3e}), mean-abs {mn:.3e}"
+    mean_bound = MEAN_ABS + 0.5 * BF16_U * float(np.abs(ref).mean())
+    assert excess.max() <= 0 and mn <= mean_bound, \
+        f"{what}: max-abs {mx:.3e} (over the bound by {excess.max():.3e}), " \
+        f"mean-abs {mn:.3e} (bound {mean_bound:.3e})"
     return mx, mn
 
 
