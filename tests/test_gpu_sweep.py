@@ -153,3 +153,33 @@ def test_sweep_varlen(swa, case):
     assert swa.swa_get_device_status() == 0
     ref = oracle.swa_varlen(q, k, v, cu, W, scale, n_sink=S)
     assert_close_bf16out(to_f64(out), ref, what=f"varlen lens{lens} H{H}/{Hkv} d{d} W{W} S{S}")
+
+
+@pytest.mark.parametrize("case", range(16))
+def test_sweep_backward(swa, case):
+    """Gradients of random small shapes, each tensor bounded by its own scale
+    (max-abs <= 8u max|ref|, mean-abs <= 2u mean|ref|, u = 2^-8)."""
+    rng, H, Hkv, d = _case(5000 + case)
+    B = int(rng.integers(1, 3))
+    N = int(rng.integers(1, 600))
+    W = int(rng.choice([1, int(rng.integers(2, 300)), N + 10]))
+    q = si.normal_bf16(case, si.STREAM["q"], (B, H, N, d))
+    k = si.normal_bf16(case, si.STREAM["k"], (B, Hkv, N, d))
+    v = si.normal_bf16(case, si.STREAM["v"], (B, Hkv, N, d))
+    g = si.normal_bf16(case, si.STREAM["extra"], (B, H, N, d))
+    scale = 1.0 / math.sqrt(d)
+    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    out, lse = swa.swa_attn_fwd(tq, tk, tv, W, scale, return_lse=True)
+    grads = swa.swa_attn_bwd(tq, tk, tv, out, to_dev(g), lse, W, scale)
+    assert swa.swa_get_device_status() == 0
+    u = 2.0 ** -8
+    for name, got, ref in zip(("dq", "dk", "dv"), grads, oracle.swa_backward(q, k, v, g, W, scale)):
+        got = to_f64(got)
+        err = np.abs(got - ref)
+        what = f"backward {name} B{B} H{H}/{Hkv} N{N} d{d} W{W}"
+        assert np.all(np.isfinite(got)), what
+        if np.abs(ref).max() == 0:  # W = 1 or a single position: exactly 0 in the oracle
+            assert err.max() < 1e-4, what
+            continue
+        assert err.max() <= 8 * u * np.abs(ref).max(), f"{what}: max-abs {err.max():.3e}"
+        assert err.mean() <= 2 * u * np.abs(ref).mean(), f"{what}: mean-abs {err.mean():.3e}"
