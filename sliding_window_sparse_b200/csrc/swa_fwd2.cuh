@@ -311,6 +311,15 @@ struct Walker2 {
   }
 };
 
+// 256-bit store of 8 words to a 32-byte-aligned global address.
+__device__ __forceinline__ void st_global_v8(void *ptr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d, uint32_t e, uint32_t f, uint32_t g,
+                                             uint32_t h) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a),
+               "r"(b), "r"(c), "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
+               : "memory");
+}
+
 template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kFwd2Threads, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -749,6 +758,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         ++u_iter;
         tc_fence_after();
         const float inv_l = 1.f / l_run;
+        const bool out32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
         const int hh = U.h[x];
         __nv_bfloat16 *orow =
             p.out + (MODE == 2 ? (qs + qrow) * p.H + hh
@@ -759,14 +769,23 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           uint32_t o32[32];
           tmem_ld32(tO + cb2 * 32, o32);
           if (qrow < len) {
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(o32[i + 0]) * inv_l, __uint_as_float(o32[i + 1]) * inv_l);
-              v.y = pack_bf16(__uint_as_float(o32[i + 2]) * inv_l, __uint_as_float(o32[i + 3]) * inv_l);
-              v.z = pack_bf16(__uint_as_float(o32[i + 4]) * inv_l, __uint_as_float(o32[i + 5]) * inv_l);
-              v.w = pack_bf16(__uint_as_float(o32[i + 6]) * inv_l, __uint_as_float(o32[i + 7]) * inv_l);
-              *reinterpret_cast<uint4 *>(orow + cb2 * 32 + i) = v;
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16(__uint_as_float(o32[2 * i]) * inv_l,
+                                __uint_as_float(o32[2 * i + 1]) * inv_l);
+            // whole 32-byte sectors when the rows allow it (each thread writes
+            // its own row, so every store of a warp touches 32 rows)
+            if (out32) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 8)
+                st_global_v8(orow + cb2 * 32 + 2 * i, pk[i], pk[i + 1], pk[i + 2], pk[i + 3],
+                             pk[i + 4], pk[i + 5], pk[i + 6], pk[i + 7]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<uint4 *>(orow + cb2 * 32 + 2 * i) =
+                    make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
             }
           }
         }
