@@ -97,6 +97,29 @@ __device__ __forceinline__ void tmem_ld_wait2(uint32_t (&a)[32], uint32_t (&b)[3
                : "memory");
 }
 
+// One 32-column chunk of a gradient row, scaled, as bf16: 64 bytes, stored as two
+// 256-bit stores (whole sectors) when the row is 32-byte aligned, else as four
+// 16-byte stores.
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16 *dst, const uint32_t (&o32)[32],
+                                                float mul, bool aligned32) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    pk[i] = pack_bf16(__uint_as_float(o32[2 * i]) * mul, __uint_as_float(o32[2 * i + 1]) * mul);
+  if (aligned32) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 8)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 2 * i),
+                   "r"(pk[i]), "r"(pk[i + 1]), "r"(pk[i + 2]), "r"(pk[i + 3]), "r"(pk[i + 4]),
+                   "r"(pk[i + 5]), "r"(pk[i + 6]), "r"(pk[i + 7])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; i += 4)
+      *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
+  }
+}
+
 // Columns [lo, hi] (clipped to the tile) as four 32-bit words.
 __device__ __forceinline__ void col_mask(int lo, int hi, uint32_t (&mw)[4]) {
 #pragma unroll
@@ -417,17 +440,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t o32[32];
         tmem_ld32(tmem + T_DQ + lane_off + cb * 32, o32);
-        if (valid) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 v;
-            v.x = pack_bf16(__uint_as_float(o32[i + 0]) * p.scale, __uint_as_float(o32[i + 1]) * p.scale);
-            v.y = pack_bf16(__uint_as_float(o32[i + 2]) * p.scale, __uint_as_float(o32[i + 3]) * p.scale);
-            v.z = pack_bf16(__uint_as_float(o32[i + 4]) * p.scale, __uint_as_float(o32[i + 5]) * p.scale);
-            v.w = pack_bf16(__uint_as_float(o32[i + 6]) * p.scale, __uint_as_float(o32[i + 7]) * p.scale);
-            *reinterpret_cast<uint4 *>(drow + cb * 32 + i) = v;
-          }
-        }
+        if (valid)
+          store_row_chunk(drow + cb * 32, o32, p.scale,
+                          (reinterpret_cast<uintptr_t>(p.dq) & 31u) == 0);
       }
       tc_fence_before();
       mbar_arrive(BAR_DQE);
@@ -774,17 +789,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int cb = 0; cb < D / 32; ++cb) {
           uint32_t o32[32];
           tmem_ld32(src + cb * 32, o32);
-          if (valid) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(o32[i + 0]) * mul, __uint_as_float(o32[i + 1]) * mul);
-              v.y = pack_bf16(__uint_as_float(o32[i + 2]) * mul, __uint_as_float(o32[i + 3]) * mul);
-              v.z = pack_bf16(__uint_as_float(o32[i + 4]) * mul, __uint_as_float(o32[i + 5]) * mul);
-              v.w = pack_bf16(__uint_as_float(o32[i + 6]) * mul, __uint_as_float(o32[i + 7]) * mul);
-              *reinterpret_cast<uint4 *>(drow + cb * 32 + i) = v;
-            }
-          }
+          if (valid)
+            store_row_chunk(drow + cb * 32, o32, mul,
+                            (reinterpret_cast<uintptr_t>(which == 0 ? p.dv : p.dk) & 31u) == 0);
         }
       }
       tc_fence_before();
