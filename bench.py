@@ -569,13 +569,17 @@ def run_native(args):
                               "roofline": {"bound": "hbm", "achieved": gbs,
                                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                            "frac": gbs / peaks["hbm_gbs"],
+                                           "traffic": profiled_traffic("decode_split_kernel",
+                                                                       name),
                                            "note": "KV bytes over split+combine time"}})
             else:
                 tf = useful_flops(pw) / (pms * 1e-3) / 1e12
                 entry.update({"value": tf * world, "unit": "TFLOP/s",
                               "roofline": {"bound": "tensor", "achieved": tf,
                                            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                           "frac": tf / peaks["bf16_tflops"]}})
+                                           "frac": tf / peaks["bf16_tflops"],
+                                           "traffic": (profiled_traffic("fwd2_kernel", name)
+                                                       if pw.kind != "backward" else None)}})
             paths[name] = entry
             del px, pcall
             torch.cuda.empty_cache()
