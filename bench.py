@@ -177,7 +177,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "fwd2_kernel": ("swa_fwd2.cuh", "sm100.cuh"),
+    "fwd2_kernel": ("swa_fwd2.cuh", "swa_tile.cuh", "swa_epilogue.cuh", "sm100.cuh"),
     "decode_split_kernel": ("swa_decode.cuh", "sm100.cuh"),
 }
 

@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+#include "swa_epilogue.cuh"
 
 namespace swa {
 
@@ -95,29 +96,6 @@ __device__ __forceinline__ void tmem_ld_wait2(uint32_t (&a)[32], uint32_t (&b)[3
                : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]), "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]), "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
                :
                : "memory");
-}
-
-// One 32-column chunk of a gradient row, scaled, as bf16: 64 bytes, stored as two
-// 256-bit stores (whole sectors) when the row is 32-byte aligned, else as four
-// 16-byte stores.
-__device__ __forceinline__ void store_row_chunk(__nv_bfloat16 *dst, const uint32_t (&o32)[32],
-                                                float mul, bool aligned32) {
-  uint32_t pk[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    pk[i] = pack_bf16(__uint_as_float(o32[2 * i]) * mul, __uint_as_float(o32[2 * i + 1]) * mul);
-  if (aligned32) {
-#pragma unroll
-    for (int i = 0; i < 16; i += 8)
-      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 2 * i),
-                   "r"(pk[i]), "r"(pk[i + 1]), "r"(pk[i + 2]), "r"(pk[i + 3]), "r"(pk[i + 4]),
-                   "r"(pk[i + 5]), "r"(pk[i + 6]), "r"(pk[i + 7])
-                   : "memory");
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; i += 4)
-      *reinterpret_cast<uint4 *>(dst + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
-  }
 }
 
 // Columns [lo, hi] (clipped to the tile) as four 32-bit words.
@@ -435,14 +413,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait(BAR_DQF, u_iter & 1, abort_flag)) break;
       ++u_iter;
       tc_fence_after();
-      __nv_bfloat16 *drow = p.dq + r * D;
-#pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t o32[32];
-        tmem_ld32(tmem + T_DQ + lane_off + cb * 32, o32);
-        if (valid)
-          store_row_chunk(drow + cb * 32, o32, p.scale,
-                          (reinterpret_cast<uintptr_t>(p.dq) & 31u) == 0);
+      {
+        // rows of this lane's 8-lane group: whole 128-byte segments per store
+        const int g_row = t * kBwdT + quad * 32 + (lane & ~7);
+        store_tile_rows<D>(p.dq + ((static_cast<int64_t>(b) * p.H + h) * p.N + g_row) * D, D,
+                           p.N - g_row, tmem + T_DQ + lane_off, p.scale, lane);
       }
       tc_fence_before();
       mbar_arrive(BAR_DQE);
@@ -778,22 +753,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait(BAR_AF, u_iter & 1, abort_flag)) break;
       ++u_iter;
       tc_fence_after();
-      const bool valid = krow < p.N;
-      const int64_t r = (static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + krow;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16 *drow = (which == 0 ? p.dv : p.dk) + r * D;
-        const float mul = which == 0 ? 1.f : p.scale;
-        const uint32_t src = tmem + (which == 0 ? T_DV : T_DK) + lane_off;
-#pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t o32[32];
-          tmem_ld32(src + cb * 32, o32);
-          if (valid)
-            store_row_chunk(drow + cb * 32, o32, mul,
-                            (reinterpret_cast<uintptr_t>(which == 0 ? p.dv : p.dk) & 31u) == 0);
-        }
-      }
+      // rows of this lane's 8-lane group: whole 128-byte segments per store
+      const int g_row = kt * kBwdT + quad * 32 + (lane & ~7);
+      const int64_t g_off = ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + g_row) * D;
+      store_tile_rows<D>(p.dv + g_off, D, p.N - g_row, tmem + T_DV + lane_off, 1.f, lane);
+      store_tile_rows<D>(p.dk + g_off, D, p.N - g_row, tmem + T_DK + lane_off, p.scale, lane);
       tc_fence_before();
       mbar_arrive(BAR_AE);
     }

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+#include "swa_epilogue.cuh"
 #include "swa_tile.cuh"
 
 namespace swa {
@@ -310,33 +311,6 @@ struct Walker2 {
     return false;
   }
 };
-
-// Transpose, within each group of 8 lanes, an 8 x 8 matrix of 16-byte pieces:
-// on entry lane j of a group holds pieces 0..7 of its own row j (piece i in
-// e[4i..4i+3]); on exit it holds piece j of rows 0..7 of the group (row i's in
-// e[4i..4i+3]).  Stage s swaps bit s of the row index with bit s of the piece
-// index: the lane whose bit s is 0 keeps the pieces whose bit s is 0 and trades
-// the others with lane ^ (1 << s).
-__device__ __forceinline__ void transpose8_pieces(uint32_t (&e)[32], int lane) {
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    const int m = 1 << s;
-    const bool hi = (lane >> s) & 1;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i & m) continue;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t send = hi ? e[4 * i + w] : e[4 * (i | m) + w];
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
-        if (hi)
-          e[4 * i + w] = recv;
-        else
-          e[4 * (i | m) + w] = recv;
-      }
-    }
-  }
-}
 
 template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kFwd2Threads, 1)
@@ -777,37 +751,13 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         tc_fence_after();
         const float inv_l = 1.f / l_run;
         const int hh = U.h[x];
-        // 64 columns at a time: each thread packs its own row, the 8-lane groups
-        // transpose 16-byte pieces, and each store instruction then writes four
-        // whole 128-byte row segments (8 lanes per segment) instead of 32 rows'
-        // scattered sectors
+        // rows of this lane's 8-lane group: whole 128-byte segments per store
         const int grp_row = U.t[x] * kQT + quad * 32 + (lane & ~7);
-        const int64_t row_stride = MODE == 2 ? static_cast<int64_t>(p.H) * D : D;
-        __nv_bfloat16 *gptr =
+        store_tile_rows<D>(
             p.out + (MODE == 2 ? (qs + grp_row) * p.H + hh
                                : static_cast<int64_t>(U.b * p.H + hh) * p.n_q + grp_row) *
-                        static_cast<int64_t>(D) +
-            8 * (lane & 7);
-        const int n_valid = len - grp_row;  // rows of this lane group inside the output
-#pragma unroll 1
-        for (int h2 = 0; h2 < D / 64; ++h2) {
-          uint32_t e[32];
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t o32[32];
-            tmem_ld32(tO + h2 * 64 + c2 * 32, o32);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              e[c2 * 16 + i] = pack_bf16(__uint_as_float(o32[2 * i]) * inv_l,
-                                         __uint_as_float(o32[2 * i + 1]) * inv_l);
-          }
-          transpose8_pieces(e, lane);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (i < n_valid)
-              *reinterpret_cast<uint4 *>(gptr + i * row_stride + h2 * 64) =
-                  make_uint4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]);
-        }
+                        static_cast<int64_t>(D),
+            MODE == 2 ? static_cast<int64_t>(p.H) * D : D, len - grp_row, tO, inv_l, lane);
         if (p.lse && qrow < len)
           p.lse[MODE == 2 ? static_cast<int64_t>(hh) * p.total + qs + qrow
                           : static_cast<int64_t>(U.b * p.H + hh) * p.n_q + qrow] =
