@@ -5,7 +5,11 @@ max(0, i - W + 1) .. i (the window includes the query's own position), and
 the softmax is taken over those pairs only.  Every step runs in the CUDA
 kernels of ``libswa.so`` behind the C ABI of ``include/swa.h``; this module
 only marshals torch tensors (device memory, current stream) into those calls.
-The function names match the C entry points.
+The function names match the C entry points.  One addition sits above them:
+``swa_attn_fwd_seq_parallel`` (module ``seq_parallel``) splits a sequence
+along its length across ``torch.distributed`` ranks; it exchanges the W - 1
+key/value rows before each shard and then calls ``swa_ring_write`` and
+``swa_attn_chunk_ring``.
 
 Layouts (row-major bf16): queries ``[B, H, rows, d]``, keys/values
 ``[B, Hkv, rows, d]``, ring caches ``[B, Hkv, W, d]``; query head h reads
@@ -39,6 +43,7 @@ __all__ = [
     "swa_ring_slot_positions",
     "swa_get_device_status",
     "swa_version",
+    "swa_attn_fwd_seq_parallel",
 ]
 
 
@@ -356,3 +361,12 @@ def swa_get_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word as a status code."""
     s = _stream() if stream is None else stream
     return int(lib().swa_get_device_status(s))
+
+
+def swa_attn_fwd_seq_parallel(q, k, v, W: int, scale: float | None = None, out=None,
+                              return_lse: bool = False, group=None, ring_k=None, ring_v=None):
+    """Prefill of a sequence split along its length across ranks (see ``seq_parallel``)."""
+    from .seq_parallel import swa_attn_fwd_seq_parallel as run
+
+    return run(q, k, v, W, scale=scale, out=out, return_lse=return_lse, group=group,
+               ring_k=ring_k, ring_v=ring_v)
