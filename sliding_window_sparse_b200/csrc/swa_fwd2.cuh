@@ -8,7 +8,7 @@
 // windows and each tile uses its own part).  CTAs are persistent and walk the
 // heavy-first unit order in a serpentine (see unit_of).
 //
-// Roles (320 threads):
+// Roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q_A, Q_B once per unit, then K and V tiles into
 //               separate shared-memory rings (3 K and 2 V stages at d = 128;
 //               128-byte swizzle, one box per 64 head-dim columns).  Only live
@@ -18,7 +18,8 @@
 //                 O_X += P_X V         (P from tensor memory, V from shared memory)
 //               in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
 //               softmax of one tile overlaps the MMAs of the other.
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one row per
+//   warps 2-3   idle (they complete warpgroup 0).
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one row per
 //               thread, one tensor-memory lane quadrant per warp.  Mask only
 //               partial or ragged tiles, base-2 exponentials with
 //               scale * log2(e) folded in, running max and sum in fp32, P
@@ -26,6 +27,14 @@
 //               memory only when the running max grows by more than 2^8.
 //               After the unit's last tile: O / l to bf16 rows, and the
 //               log-sum-exp.
+//
+// Registers: 384 threads get 168 registers each at launch (three warps per
+// SM sub-partition).  Warpgroup 0 then gives registers back (setmaxnreg.dec to
+// kRegsControl) and the two softmax warpgroups take them (setmaxnreg.inc to
+// kRegsSoftmax), so the softmax holds a whole 128-column score row without
+// spilling.  The split must add up to the launch total exactly, or the
+// increase would wait for registers that never come: the host checks the
+// kernel's launch register count before the first launch.
 //
 // Tensor memory (512 columns): S_A/P_A [0,128), S_B/P_B [128,256),
 // O_A [256, 256+D), O_B [256+D, 256+2D).  P_X overwrites the first 64 columns
@@ -44,7 +53,14 @@ namespace swa {
 
 constexpr int kQT = 128;  // query rows per tile (MMA M, tensor-memory lanes)
 constexpr int kKT = 128;  // keys per tile
-constexpr int kFwd2Threads = 320;
+constexpr int kFwd2Threads = 384;
+constexpr int kFwd2LaunchRegs = 168;  // registers per thread at launch (checked by the host)
+constexpr int kRegsControl = 88;      // warpgroup 0: producer, MMA issuer, two idle warps
+constexpr int kRegsSoftmax = 208;     // warpgroups 1 and 2: softmax + epilogue
+static_assert(4 * kRegsControl + 8 * kRegsSoftmax == (kFwd2Threads / 32) * kFwd2LaunchRegs,
+              "the register split must hand over exactly the launch allocation");
+static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0 && kRegsSoftmax <= 256,
+              "setmaxnreg counts are multiples of 8, at most 256");
 constexpr float kLazyRescaleLog2 = 8.0f;
 // The exponentials of the last kEmuCols columns of every tile are evaluated
 // on the FMA pipe (ex2_poly2) instead of the MUFU, to balance the two pipes.
@@ -312,6 +328,16 @@ struct Walker2 {
   }
 };
 
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kFwd2Threads, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -417,6 +443,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     return 0;
   };
 
+  if (warp < 4) {
+  warpgroup_regs_dec<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -591,9 +619,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         ++q_iter;
       }
     }
+  }  // warps 2 and 3 have no role
   } else {
+    warpgroup_regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax + epilogue
-    const int x = warp < 6 ? 0 : 1;  // query tile of this warp group
+    const int x = warp < 8 ? 0 : 1;  // query tile of this warp group
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;

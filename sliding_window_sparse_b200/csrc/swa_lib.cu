@@ -109,6 +109,15 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
       cudaSuccess)
     return SWA_ERR_CUDA;
+  // The kernel's warpgroups re-split the registers it is launched with
+  // (setmaxnreg); that split assumes exactly kFwd2LaunchRegs per thread.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SWA_ERR_CUDA;
+    launch_regs = fa.numRegs;
+  }
+  if (launch_regs != swa::kFwd2LaunchRegs) return SWA_ERR_UNSUPPORTED;
   p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
   const int64_t units = p.pair_heads
                             ? static_cast<int64_t>(p.B) * p.Hkv * (p.G / 2) * p.nqt
