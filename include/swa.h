@@ -29,8 +29,14 @@
  *    anything is enqueued: an invalid argument enqueues nothing.  Errors found
  *    on the device (a negative position, a wait that timed out) set a device
  *    status word that swa_get_device_status() reads and clears.
- *  - Thread safety: calls are stateless apart from a per-process cache of a
- *    driver entry point, which is set up once under a lock.
+ *  - Thread safety: calls are stateless apart from per-process caches: a
+ *    driver entry point (set up once under a lock) and the launch register
+ *    count of each attention-kernel variant (read once; every thread reads
+ *    the same value).
+ *  - The prefill / chunk / varlen kernels re-split their registers between
+ *    warp groups and are written for 168 registers per thread at launch; a
+ *    build that compiled them otherwise makes those calls return
+ *    SWA_ERR_UNSUPPORTED instead of launching.
  */
 #ifndef SWA_H_
 #define SWA_H_
