@@ -31,6 +31,10 @@ Functions and the passages they follow (page title, section):
 * :func:`swa_backward`    -- M003 note sections 07-08 (Q/K/V gradients under the
                              same mask); :func:`swa_forward_f64` is the forward
                              on fp64 inputs that its finite differences use.
+* :func:`swa_varlen_backward` -- the same gradients for packed sequences with
+                             optional sinks (blog section 5.2 tip 4, taxonomy
+                             page section 3.2); :func:`swa_varlen_f64` is its
+                             fp64 forward.
 
 All of them are pinned by ``tests/test_oracle_pins.py``.
 """
@@ -116,6 +120,12 @@ def _configure(lib):
     lib.orc_swa_backward.restype = _i64
     lib.orc_swa_backward.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _i64, _int, _i64,
                                      _dbl, _ptr, _ptr, _ptr]
+    lib.orc_swa_varlen_f64.restype = _i64
+    lib.orc_swa_varlen_f64.argtypes = [_ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int, _i64,
+                                       _i64, _dbl, _ptr]
+    lib.orc_swa_varlen_backward.restype = _i64
+    lib.orc_swa_varlen_backward.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _int, _int, _int, _int,
+                                            _i64, _i64, _dbl, _ptr, _ptr, _ptr]
     lib.orc_tile_classes.restype = _int
     lib.orc_tile_classes.argtypes = [_int, _int, _i64, _i64, _ptr, _i64, _int, _int, _ptr,
                                      _ptr]
@@ -267,6 +277,50 @@ def swa_backward(q, k, v, dout, W: int, scale: float):
     if _load().orc_swa_backward(_p(q), _p(k), _p(v), _p(dout), B, H, Hkv, N, d, W, scale,
                                 _p(dq), _p(dk), _p(dv)):
         raise ValueError("query rows without a legal key")
+    return dq, dk, dv
+
+
+def _cu(cu_seqlens, total):
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64).reshape(-1)
+    if cu[-1] != total:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    return cu
+
+
+def swa_varlen_f64(q, k, v, cu_seqlens, W: int, scale: float, n_sink: int = 0):
+    """swa_varlen on fp64 inputs (the function the varlen gradient pins differentiate).
+
+    q: [total,H,d], k/v: [total,Hkv,d]; bf16 bits or float arrays.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    total, H, d = q.shape
+    cu = _cu(cu_seqlens, total)
+    out = np.empty((total, H, d), dtype=np.float64)
+    bad = _load().orc_swa_varlen_f64(_p(q), _p(k), _p(v), _p(cu), cu.shape[0] - 1, H,
+                                     k.shape[1], d, W, n_sink, scale, _p(out))
+    if bad:
+        raise ValueError("malformed cu_seqlens" if bad < 0 else "query rows without a legal key")
+    return out
+
+
+def swa_varlen_backward(q, k, v, dout, cu_seqlens, W: int, scale: float, n_sink: int = 0):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the packed varlen prefill
+    (per-sequence windows, optional sinks), in fp64.
+
+    q, dout: [total,H,d]; k, v: [total,Hkv,d]; bf16 bits or float arrays.
+    """
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    total, H, d = q.shape
+    Hkv = k.shape[1]
+    cu = _cu(cu_seqlens, total)
+    dq = np.empty((total, H, d), dtype=np.float64)
+    dk = np.empty((total, Hkv, d), dtype=np.float64)
+    dv = np.empty((total, Hkv, d), dtype=np.float64)
+    bad = _load().orc_swa_varlen_backward(_p(q), _p(k), _p(v), _p(dout), _p(cu),
+                                          cu.shape[0] - 1, H, Hkv, d, W, n_sink, scale,
+                                          _p(dq), _p(dk), _p(dv))
+    if bad:
+        raise ValueError("malformed cu_seqlens" if bad < 0 else "query rows without a legal key")
     return dq, dk, dv
 
 

@@ -787,3 +787,154 @@ int orc_tile_classes(int mode, int B, int64_t n_q, int64_t n_k, const int64_t *q
     free(kpos);
     return 0;
 }
+
+/* cu_seqlens starts at 0 and never decreases; returns the longest sequence,
+ * or -1 when malformed. */
+static int64_t varlen_longest(const int64_t *cu_seqlens, int n_seq)
+{
+    if (cu_seqlens[0] != 0) return -1;
+    int64_t longest = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (len < 0) return -1;
+        if (len > longest) longest = len;
+    }
+    return longest;
+}
+
+/*
+ * Packed variable-length forward on fp64 inputs ([BLOG s5.2] tip 4, with the
+ * sink rule of [TAXO s3.2]): the function whose finite differences pin
+ * orc_swa_varlen_backward.  q, out: [total, H, d]; k, v: [total, Hkv, d].
+ * Sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1] - 1 at positions
+ * 0, 1, ...; its token i reads the keys j of the same sequence with
+ * allowed_sink(i, j, W, S), in increasing j (two-pass softmax as in
+ * orc_swa_forward_f64).  Returns -1 for malformed cu_seqlens, else the number
+ * of rows with no legal key.
+ */
+int64_t orc_swa_varlen_f64(const double *q, const double *k, const double *v,
+                           const int64_t *cu_seqlens, int n_seq, int H, int Hkv, int d,
+                           int64_t W, int64_t S, double scale, double *out)
+{
+    int64_t longest = varlen_longest(cu_seqlens, n_seq);
+    if (longest < 0) return -1;
+    int64_t bad = 0;
+    double *sc = (double *)malloc(sizeof(double) * (size_t)(longest > 0 ? longest : 1));
+    int64_t *idx = (int64_t *)malloc(sizeof(int64_t) * (size_t)(longest > 0 ? longest : 1));
+    for (int s = 0; s < n_seq; ++s) {
+        int64_t first = cu_seqlens[s], len = cu_seqlens[s + 1] - first;
+        for (int64_t h = 0; h < H; ++h) {
+            int64_t kh = kv_head(h, H, Hkv);
+            for (int64_t i = 0; i < len; ++i) {
+                const double *qi = q + ((first + i) * H + h) * d;
+                double *o = out + ((first + i) * H + h) * d;
+                int64_t n = 0;
+                for (int64_t j = 0; j < len; ++j)
+                    if (allowed_sink(i, j, W, S)) idx[n++] = j;
+                if (n == 0) { ++bad; continue; }
+                double smax = -INFINITY;
+                for (int64_t t = 0; t < n; ++t) {
+                    const double *kj = k + ((first + idx[t]) * Hkv + kh) * d;
+                    double x = 0.0;
+                    for (int c = 0; c < d; ++c) x += qi[c] * kj[c];
+                    sc[t] = x * scale;
+                    if (sc[t] > smax) smax = sc[t];
+                }
+                double denom = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    sc[t] = exp(sc[t] - smax);
+                    denom += sc[t];
+                }
+                for (int c = 0; c < d; ++c) o[c] = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    const double *vj = v + ((first + idx[t]) * Hkv + kh) * d;
+                    for (int c = 0; c < d; ++c) o[c] += sc[t] / denom * vj[c];
+                }
+            }
+        }
+    }
+    free(sc);
+    free(idx);
+    return bad;
+}
+
+/*
+ * Gradients of the packed variable-length forward, sinks included ([M003
+ * s07-s08]: Q/K/V gradients under the same mask as the output; the mask is
+ * that of orc_swa_varlen_f64).  For the loss sum(out * dout), per sequence:
+ *   P_ij  = softmax over the visible j of scale * <q_i, k_j>
+ *   dP_ij = <dout_i, v_j>,   D_i = sum_j P_ij dP_ij,   dS_ij = P_ij (dP_ij - D_i)
+ *   dq_i  = scale * sum_j dS_ij k_j
+ *   dk_j  = scale * sum_i dS_ij q_i   (over the query heads of j's group)
+ *   dv_j  = sum_i P_ij dout_i         (likewise)
+ * q, dout, dq: [total, H, d]; k, v, dk, dv: [total, Hkv, d]; fp64.
+ * Returns -1 for malformed cu_seqlens, else the number of rows with no legal key.
+ */
+int64_t orc_swa_varlen_backward(const double *q, const double *k, const double *v,
+                                const double *dout, const int64_t *cu_seqlens, int n_seq,
+                                int H, int Hkv, int d, int64_t W, int64_t S, double scale,
+                                double *dq, double *dk, double *dv)
+{
+    int64_t longest = varlen_longest(cu_seqlens, n_seq);
+    if (longest < 0) return -1;
+    int64_t total = cu_seqlens[n_seq];
+    memset(dq, 0, sizeof(double) * (size_t)(total * H * d));
+    memset(dk, 0, sizeof(double) * (size_t)(total * Hkv * d));
+    memset(dv, 0, sizeof(double) * (size_t)(total * Hkv * d));
+    int64_t bad = 0;
+    int64_t cap = longest > 0 ? longest : 1;
+    double *p = (double *)malloc(sizeof(double) * (size_t)cap);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)cap);
+    int64_t *idx = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+    for (int s = 0; s < n_seq; ++s) {
+        int64_t first = cu_seqlens[s], len = cu_seqlens[s + 1] - first;
+        for (int64_t h = 0; h < H; ++h) {
+            int64_t kh = kv_head(h, H, Hkv);
+            for (int64_t i = 0; i < len; ++i) {
+                const double *qi = q + ((first + i) * H + h) * d;
+                const double *gi = dout + ((first + i) * H + h) * d;
+                int64_t n = 0;
+                for (int64_t j = 0; j < len; ++j)
+                    if (allowed_sink(i, j, W, S)) idx[n++] = j;
+                if (n == 0) { ++bad; continue; }
+                double smax = -INFINITY;
+                for (int64_t t = 0; t < n; ++t) {
+                    const double *kj = k + ((first + idx[t]) * Hkv + kh) * d;
+                    double x = 0.0;
+                    for (int c = 0; c < d; ++c) x += qi[c] * kj[c];
+                    p[t] = x * scale;
+                    if (p[t] > smax) smax = p[t];
+                }
+                double denom = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    p[t] = exp(p[t] - smax);
+                    denom += p[t];
+                }
+                double Di = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    const double *vj = v + ((first + idx[t]) * Hkv + kh) * d;
+                    p[t] /= denom;
+                    double g = 0.0;
+                    for (int c = 0; c < d; ++c) g += gi[c] * vj[c];
+                    dp[t] = g;
+                    Di += p[t] * g;
+                }
+                double *dqi = dq + ((first + i) * H + h) * d;
+                for (int64_t t = 0; t < n; ++t) {
+                    double ds = p[t] * (dp[t] - Di);
+                    int64_t row = (first + idx[t]) * Hkv + kh;
+                    const double *kj = k + row * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqi[c] += scale * ds * kj[c];
+                        dk[row * d + c] += scale * ds * qi[c];
+                        dv[row * d + c] += p[t] * gi[c];
+                    }
+                }
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    free(idx);
+    return bad;
+}

@@ -3,7 +3,7 @@
 Each mutant is a copy of oracle/swa_oracle.c with one planted mistake (an
 off-by-one window, a flipped causal bound, a dropped scale or denominator, a
 transposed operand, a wrong head map, a wrong ring or chunk index, a swapped
-tile class, ...), compiled into a temporary directory.  The pins of
+tile class, a gradient without its D term, ...), compiled into a temporary directory.  The pins of
 tests/test_oracle_pins.py run against the mutant through oracle.use_library;
 every mutant must make at least one of them fail.  The committed oracle is
 never modified.
@@ -58,6 +58,16 @@ MUTANTS = {
     "backward_dk_unscaled": ("dkj[c] += scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
     "backward_dv_from_q": ("dvj[c] += p[j - lo] * gi[c];", "dvj[c] += p[j - lo] * qi[c];"),
     "backward_dq_from_q": ("dqi[c] += scale * ds * kj[c];", "dqi[c] += scale * ds * qi[c];"),
+    "varlen_backward_delta_dropped": ("double ds = p[t] * (dp[t] - Di);",
+                                      "double ds = p[t] * dp[t];"),
+    "varlen_backward_dk_unscaled": ("dk[row * d + c] += scale * ds * qi[c];",
+                                    "dk[row * d + c] += ds * qi[c];"),
+    "varlen_backward_dv_from_q": ("dv[row * d + c] += p[t] * gi[c];",
+                                  "dv[row * d + c] += p[t] * qi[c];"),
+    "varlen_backward_sequence_base_dropped": ("int64_t row = (first + idx[t]) * Hkv + kh;",
+                                              "int64_t row = idx[t] * Hkv + kh;"),
+    "varlen_f64_sinks_ignored": ("if (allowed_sink(i, j, W, S)) idx[n++] = j;",
+                                 "if (allowed(i, j, W)) idx[n++] = j;"),
 }
 
 
@@ -98,6 +108,11 @@ def _pin_suite(golden_dir):
         lambda: pins.test_backward_finite_differences(3),
         lambda: pins.test_backward_full_window_equals_torch_autograd(1, 4, 2, 37, 16),
         lambda: pins.test_backward_window_one(),
+        lambda: pins.test_varlen_backward_finite_differences(3, 2),
+        lambda: pins.test_varlen_backward_equals_dense_mask_autograd([7, 3, 12], 4, 2),
+        lambda: pins.test_varlen_backward_single_sequence_equals_linear(),
+        lambda: pins.test_varlen_backward_no_cross_talk(),
+        lambda: pins.test_varlen_backward_window_one(),
     ]
 
 

@@ -651,6 +651,111 @@ def test_backward_window_one():
     assert np.max(np.abs(dv - want)) < 1e-14
 
 
+# --- gradients of the packed varlen prefill with sinks ------------------------
+
+def _packed_f64(seed, lens, H, Hkv, d):
+    total = int(sum(lens))
+
+    def draw(shape, stream):
+        return si.bf16_bits_to_f32(_rand(seed, shape, si.STREAM[stream])).astype(np.float64)
+
+    q, g = draw((total, H, d), "q"), draw((total, H, d), "extra")
+    k, v = draw((total, Hkv, d), "k"), draw((total, Hkv, d), "v")
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return q, k, v, g, cu
+
+
+@pytest.mark.parametrize("W,S", [(3, 0), (3, 2), (1, 1), (100, 0)])
+def test_varlen_backward_finite_differences(W, S):
+    """Central differences of L = sum(out * g) through the fp64 varlen forward."""
+    lens, H, Hkv, d, scale = [5, 1, 6], 2, 1, 4, 0.7
+    q, k, v, g, cu = _packed_f64(40, lens, H, Hkv, d)
+    dq, dk, dv = oracle.swa_varlen_backward(q, k, v, g, cu, W, scale, n_sink=S)
+
+    def loss():
+        return float(np.sum(oracle.swa_varlen_f64(q, k, v, cu, W, scale, n_sink=S) * g))
+
+    h = 1e-5
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            up = loss()
+            x[idx] = old - h
+            dn = loss()
+            x[idx] = old
+            fd[idx] = (up - dn) / (2 * h)
+        assert np.max(np.abs(fd - grad)) < 1e-7, name
+
+
+@pytest.mark.parametrize("lens,W,S", [([7, 3, 12], 4, 2), ([9, 9], 2, 0), ([16], 5, 3),
+                                      ([4, 1, 8, 2], 100, 0)])
+def test_varlen_backward_equals_dense_mask_autograd(lens, W, S):
+    """torch fp64 autograd through a dense masked softmax per sequence, the mask
+    being the pages' rule: key j visible to i iff j <= i and (i - j < W or j < S)."""
+    import torch
+
+    H, Hkv, d, scale = 4, 2, 8, 0.35
+    q, k, v, g, cu = _packed_f64(41, lens, H, Hkv, d)
+    tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k, v))
+    loss = 0.0
+    for s, n in enumerate(lens):
+        a, b = int(cu[s]), int(cu[s + 1])
+        i = torch.arange(n).view(-1, 1)
+        j = torch.arange(n).view(1, -1)
+        visible = (j <= i) & ((i - j < W) | (j < S))
+        qs = tq[a:b].transpose(0, 1)                                    # [H, n, d]
+        ks = tk[a:b].transpose(0, 1).repeat_interleave(H // Hkv, dim=0)
+        vs = tv[a:b].transpose(0, 1).repeat_interleave(H // Hkv, dim=0)
+        sc = (qs @ ks.transpose(1, 2)) * scale
+        sc = sc.masked_fill(~visible, float("-inf"))
+        out = torch.softmax(sc, dim=-1) @ vs                            # [H, n, d]
+        loss = loss + (out.transpose(0, 1) * torch.from_numpy(g[a:b])).sum()
+    loss.backward()
+    dq, dk, dv = oracle.swa_varlen_backward(q, k, v, g, cu, W, scale, n_sink=S)
+    assert np.max(np.abs(dq - tq.grad.numpy())) < 1e-12
+    assert np.max(np.abs(dk - tk.grad.numpy())) < 1e-12
+    assert np.max(np.abs(dv - tv.grad.numpy())) < 1e-12
+
+
+def test_varlen_backward_single_sequence_equals_linear():
+    """One sequence without sinks is the linear prefill: same gradients."""
+    N, H, Hkv, d, W, scale = 20, 4, 2, 8, 6, 0.5
+    q, k, v, g, cu = _packed_f64(42, [N], H, Hkv, d)
+    dq, dk, dv = oracle.swa_varlen_backward(q, k, v, g, cu, W, scale)
+    lq, lk, lv = oracle.swa_backward(q.transpose(1, 0, 2)[None], k.transpose(1, 0, 2)[None],
+                                     v.transpose(1, 0, 2)[None], g.transpose(1, 0, 2)[None],
+                                     W, scale)
+    assert np.max(np.abs(dq - lq[0].transpose(1, 0, 2))) < 1e-13
+    assert np.max(np.abs(dk - lk[0].transpose(1, 0, 2))) < 1e-13
+    assert np.max(np.abs(dv - lv[0].transpose(1, 0, 2))) < 1e-13
+
+
+def test_varlen_backward_no_cross_talk():
+    """Changing one sequence leaves the other sequences' gradients bit-identical."""
+    lens, H, Hkv, d, W, S = [6, 4, 7], 2, 2, 4, 3, 1
+    q, k, v, g, cu = _packed_f64(43, lens, H, Hkv, d)
+    a = oracle.swa_varlen_backward(q, k, v, g, cu, W, 0.5, n_sink=S)
+    lo, hi = int(cu[1]), int(cu[2])
+    for x in (q, k, v, g):
+        x[lo:hi] *= -1.7
+    b = oracle.swa_varlen_backward(q, k, v, g, cu, W, 0.5, n_sink=S)
+    for ga, gb in zip(a, b):
+        assert np.array_equal(ga[:lo], gb[:lo]) and np.array_equal(ga[hi:], gb[hi:])
+        assert not np.array_equal(ga[lo:hi], gb[lo:hi])
+
+
+def test_varlen_backward_window_one():
+    """W = 1 without sinks: out = v, so dq = dk = 0 and dv sums dout over the group."""
+    lens, H, Hkv, d = [5, 3], 6, 2, 4
+    q, k, v, g, cu = _packed_f64(44, lens, H, Hkv, d)
+    dq, dk, dv = oracle.swa_varlen_backward(q, k, v, g, cu, 1, 0.5)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    want = g.reshape(-1, Hkv, H // Hkv, d).sum(axis=2)
+    assert np.max(np.abs(dv - want)) < 1e-14
+
+
 # --- the generator itself ------------------------------------------------------
 
 def test_generator_reproducible_and_normal():
