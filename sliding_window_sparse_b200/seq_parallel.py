@@ -70,7 +70,9 @@ def exchange_halo(k: torch.Tensor, v: torch.Tensor, W: int, group=None):
     with halo rows ``[B, Hkv, h, d]`` for positions ``start - h .. start - 1``,
     h = min(W - 1, start).  One all-gather of the shard lengths, then one
     batch of sends and receives.  Works on any backend whose point-to-point
-    ops accept the tensors' device (NCCL for CUDA tensors, gloo for CPU).
+    ops accept the tensors' device (NCCL for CUDA tensors, gloo for CPU);
+    with NCCL, set each rank's current CUDA device before the first call.
+    Every rank of the group must call it with the same W.
     """
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     B, Hkv, n, d = k.shape
