@@ -13,7 +13,9 @@ the same examples) and check that the oracle's independent paths agree:
 * packed sequences equal separate prefills of each sequence (blog section
   5.2 tip 4: windows never cross a sequence boundary);
 * the benchmark's closed-form pair count equals the enumeration, sinks
-  included (taxonomy page section 3.2).
+  included (taxonomy page section 3.2);
+* with sinks, chunks over a ring and decode both equal the one-pass packed
+  prefill with the same sinks.
 """
 
 import os
@@ -108,3 +110,48 @@ def test_packed_sequences_equal_separate_prefills(seed, lens, W, hk):
 @given(N=st.integers(1, 120), W=st.integers(1, 130), S=st.integers(0, 10))
 def test_closed_form_pairs_equal_enumeration(N, W, S):
     assert bench.sequence_pairs(N, W, S) == oracle.count_pairs_sink(N, W, S)
+
+
+@SETTINGS
+@given(seed=st.integers(0, 10_000), N=st.integers(2, 60), W=st.integers(1, 20),
+       S=st.integers(1, 6), cuts=st.lists(st.integers(1, 59), max_size=4))
+def test_chunked_with_sinks_equals_one_pass(seed, N, W, S, cuts):
+    """Chunks over a ring plus sink rows equal the one-pass prefill with the same
+    sinks (taxonomy page section 3.2 on Chapter 10 section 10.2)."""
+    B, H, Hkv, d = 1, 2, 1, 8
+    S = min(S, N)
+    q, k, v = _qkv(seed, B, H, Hkv, N, d)
+    tm = lambda x: np.ascontiguousarray(x[0].transpose(1, 0, 2))
+    full = oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, 0.45, n_sink=S).transpose(1, 0, 2)
+    sk = np.ascontiguousarray(k[:, :, :S])
+    sv = np.ascontiguousarray(v[:, :, :S])
+    rk = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rv = np.zeros_like(rk)
+    bounds = sorted({c for c in cuts if c < N} | {0, N})
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        sl = (slice(None), slice(None), slice(a, e))
+        qc, kc, vc = (np.ascontiguousarray(x[sl]) for x in (q, k, v))
+        out = oracle.swa_chunk_sink(qc, kc, vc, rk, rv, sk, sv, [a], W, 0.45)
+        assert np.array_equal(out[0], full[:, a:e])
+        rk, rv = oracle.ring_update(kc, vc, rk, rv, [a], W)
+
+
+@SETTINGS
+@given(seed=st.integers(0, 10_000), P=st.integers(0, 60), W=st.integers(1, 30),
+       S=st.integers(0, 6))
+def test_decode_with_sinks_equals_prefill_row(seed, P, W, S):
+    B, H, Hkv, d = 1, 4, 2, 8
+    N = P + 1
+    q, k, v = _qkv(seed, B, H, Hkv, N, d)
+    rk = np.zeros((B, Hkv, W, d), dtype=np.uint16)
+    rv = np.zeros_like(rk)
+    rk, rv = oracle.ring_update(k, v, rk, rv, [0], W)
+    sk = np.zeros((B, Hkv, S, d), dtype=np.uint16)
+    sv = np.zeros_like(sk)
+    n_s = min(S, N)
+    sk[:, :, :n_s] = k[:, :, :n_s]
+    sv[:, :, :n_s] = v[:, :, :n_s]
+    dec = oracle.swa_decode_sink(np.ascontiguousarray(q[:, :, P]), rk, rv, sk, sv, [P], W, 0.4)
+    tm = lambda x: np.ascontiguousarray(x[0].transpose(1, 0, 2))
+    full = oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, 0.4, n_sink=S)
+    assert np.array_equal(dec[0], full[P])
