@@ -8,9 +8,9 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dout
 // with dK and dV summed over the G query heads of a KV head.
 //
-// Two persistent kernels, each shaped like the forward: one thread issues the
-// MMAs, one feeds TMA, four warps (one 128-row tile, a row per thread) do the
-// element-wise work between the MMAs in tensor memory.
+// Two persistent kernels with the forward's roles, 192 threads each: one
+// thread issues the MMAs, one feeds TMA, four warps (one 128-row tile, a row
+// per thread) do the element-wise work between the MMAs in tensor memory.
 //
 //  * bwd_dq_kernel: one query tile of one head per unit.  Per live key tile:
 //    S = Q K^T and dP = dO V^T on the tensor cores, dS = P o (dP - D) in
