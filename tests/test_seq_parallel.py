@@ -147,3 +147,40 @@ def test_gloo_halo_exchange_and_ring_layout(tmp_path):
                                  ring_k, ring_v, np.full(B, start, np.int64), W, scale)
         ref = full.reshape(B, H, -1, D)[:, :, start:s1]
         assert np.abs(shard.reshape(ref.shape) - ref).max() <= 1e-12
+
+
+def _subgroup_main(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    from sliding_window_sparse_b200.seq_parallel import exchange_halo
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        members = [1, 2, 3]            # global rank 0 takes no part in the exchange
+        group = dist.new_group(members)
+        if rank in members:
+            lengths = [6, 3, 10]       # shard of group rank r = members.index(rank)
+            gr = members.index(rank)
+            q, k, v = _full_inputs()
+            s0 = sum(lengths[:gr])
+            k_loc = _bits_to_torch(k[:, :, s0:s0 + lengths[gr]])
+            v_loc = _bits_to_torch(v[:, :, s0:s0 + lengths[gr]])
+            start, hk, hv = exchange_halo(k_loc, v_loc, W, group=group)
+            np.save(os.path.join(out_dir, f"g_hk{gr}.npy"), _torch_to_bits(hk))
+            with open(os.path.join(out_dir, f"g_start{gr}.txt"), "w") as f:
+                f.write(str(start))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_halo_exchange_in_a_subgroup(tmp_path):
+    """Group ranks are mapped to global ranks for the point-to-point sends."""
+    world, port = 4, _free_port()
+    mp.spawn(_subgroup_main, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    _, k, _ = _full_inputs()
+    for gr, start in enumerate([0, 6, 9]):
+        assert int(open(tmp_path / f"g_start{gr}.txt").read()) == start
+        h = min(W - 1, start)
+        assert np.array_equal(np.load(tmp_path / f"g_hk{gr}.npy"), k[:, :, start - h:start])
