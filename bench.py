@@ -46,6 +46,8 @@ from swa_inputs.workloads import WORKLOADS  # noqa: E402
 FLUSH_BYTES = 256 << 20  # > 126 MB L2: written between timed steps
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 HEADLINE = "mistral_prefill"
+# workloads whose "paths" entry also times the oracle on a sample (rank 0, one GPU)
+CPU_BASELINE_PATHS = ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring")
 METRIC = "SWA prefill useful TFLOP/s and decode KV GB/s at 1 B200, % of roofline"
 
 
@@ -419,7 +421,9 @@ def time_e2e(w, x, swa, steps, warmup):
 # ----------------------------------------------------------------------------- oracle timing
 
 def oracle_sample(w, host_inputs, n_rows, seed=12345):
-    """Time the oracle on n_rows sampled query rows of workload w; returns (seconds, flops)."""
+    """Time the oracle on a sample of workload w: n_rows random query rows (prefill,
+    chunk) or n_rows sequences (decode).  Returns (seconds, work) with work in the
+    workload's unit: useful FLOPs, or K/V bytes read for decode."""
     import oracle
 
     rng = np.random.default_rng(seed)
@@ -432,24 +436,72 @@ def oracle_sample(w, host_inputs, n_rows, seed=12345):
         dt = time.perf_counter() - t0
         pairs = sum(valid_pairs_row(int(i), w.W) for i in rows[:, 2])
         return dt, 4 * w.d * pairs
+    if w.kind == "chunk" and not w.len_hi and not w.n_sink:
+        q, kn, vn, rk, rv, qs = host_inputs
+        rows = np.stack([rng.integers(w.B, size=n_rows), rng.integers(w.H, size=n_rows),
+                         rng.integers(w.Tq, size=n_rows)], axis=1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.swa_chunk(q, kn, vn, rk, rv, qs, w.W, w.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        pairs = sum(valid_pairs_row(int(qs[b]) + int(t), w.W) for b, _, t in rows)
+        return dt, 4 * w.d * pairs
+    if w.kind == "decode" and not w.n_sink:
+        q, rk, rv, pos = host_inputs
+        sel = np.sort(rng.choice(w.B, size=min(n_rows, w.B), replace=False))
+        args = [np.ascontiguousarray(a[sel]) for a in (q, rk, rv)]
+        t0 = time.perf_counter()
+        oracle.swa_decode(*args, pos[sel], w.W, w.scale)
+        dt = time.perf_counter() - t0
+        return dt, 2 * w.Hkv * w.d * 2 * w.W * len(sel)
     raise ValueError(w.kind)
 
 
+def sample_units(w) -> int:
+    """Most sample units oracle_sample can draw: query rows, or sequences for decode."""
+    if w.kind == "decode":
+        return w.B
+    if w.kind == "chunk":
+        return w.B * w.H * w.Tq
+    return w.B * w.H * w.N
+
+
 def calibrated_oracle(w, host_inputs, seconds):
-    """Grow the row sample until one oracle pass takes about `seconds`."""
-    n = 16
+    """Grow the sample until one oracle pass takes about `seconds`."""
+    n = 16 if w.kind != "decode" else 1
     dt, fl = oracle_sample(w, host_inputs, n)
-    while dt < seconds / 4 and n < w.B * w.H * w.N:
-        n = min(w.B * w.H * w.N, int(n * max(2.0, (seconds / max(dt, 1e-3)) * 0.9)))
+    while dt < seconds / 4 and n < sample_units(w):
+        n = min(sample_units(w), int(n * max(2.0, (seconds / max(dt, 1e-3)) * 0.9)))
         dt, fl = oracle_sample(w, host_inputs, n)
     return dt, fl, n
 
 
-def host_prefill_inputs(x):
+def host_inputs_of(w, x):
+    """Host (numpy) copies of a workload's device inputs in the oracle's argument order."""
     import torch
 
-    return tuple(x[n].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-                 for n in ("q", "k", "v"))
+    def bits(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    if w.kind == "prefill":
+        return tuple(bits(x[n]) for n in ("q", "k", "v"))
+    if w.kind == "chunk":
+        return tuple(bits(x[n]) for n in ("q", "k_new", "v_new", "k_ring", "v_ring")) + \
+            (x["q_start"].cpu().numpy(),)
+    return tuple(bits(x[n]) for n in ("q", "k_ring", "v_ring")) + (x["pos"].cpu().numpy(),)
+
+
+def cpu_baseline(w, host, seconds):
+    """The oracle timed on a calibrated sample of workload w, on all host cores."""
+    import oracle
+
+    dt, work, n = calibrated_oracle(w, host, seconds)
+    if w.kind == "decode":
+        return {"value": work / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{n} random sequences of {w.name} (whole ring each), {dt:.1f} s"}
+    return {"value": work / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} random query rows of {w.name} (full window each), {dt:.1f} s"}
 
 
 # ----------------------------------------------------------------------------- arms
@@ -480,7 +532,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{HEADLINE}: B1 H32 Hkv8 N8192 d128 W4096",
+        "config": {"workload": describe(w),
                    "sample": f"{n_rows} random query rows per step, full window each"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
@@ -580,6 +632,10 @@ def run_native(args):
                                            "frac": tf / peaks["bf16_tflops"],
                                            "traffic": (profiled_traffic("fwd2_kernel", name)
                                                        if pw.kind != "backward" else None)}})
+            if (rank == 0 and world == 1 and not args.no_cpu_baseline
+                    and name in CPU_BASELINE_PATHS):
+                entry["cpu_baseline"] = cpu_baseline(pw, host_inputs_of(pw, px),
+                                                     args.cpu_seconds / 3)
             paths[name] = entry
             del px, pcall
             torch.cuda.empty_cache()
@@ -589,15 +645,8 @@ def run_native(args):
 
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline and w.kind == "prefill" and not w.n_sink:
-            import oracle
-
-            host = host_prefill_inputs(x)
-            dt, fl, n_rows = calibrated_oracle(w, host, args.cpu_seconds)
-            cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                   "kind": "oracle",
-                   "sample": f"{n_rows} random query rows of {headline} (full window each), "
-                             f"{dt:.1f} s"}
+        if world == 1 and not args.no_cpu_baseline and headline in CPU_BASELINE_PATHS:
+            cpu = cpu_baseline(w, host_inputs_of(w, x), args.cpu_seconds)
         kname = "decode_split_kernel" if w.kind == "decode" else "fwd2_kernel"
         roof = {"bound": bound, "achieved": kernel_rate, "peak": peaks[peak], "unit": unit,
                 "frac": kernel_rate / peaks[peak],
@@ -611,7 +660,7 @@ def run_native(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": describe(w) + " (one batch per rank)",
+            "config": {"workload": describe(w), "batch": "one batch per rank",
                        "work_per_step": work, "l2": "flushed by a 256 MiB write "
                        "between timed steps"},
             "roofline": roof, "cpu_baseline": cpu,

@@ -24,15 +24,17 @@
  *    and enqueues kernels on `stream`; it returns before the work finishes.
  *  - d (head dim) must be 64 or 128.  W >= 1; W >= the sequence length means
  *    plain causal attention.  `scale` must be finite and > 0.
- *  - Return value: SWA_OK or one of the error codes below.  Nothing is
- *    printed and no exception crosses the ABI.  Arguments are checked before
+ *  - Return value: SWA_OK (0) or one of the positive error codes below, so
+ *    that a caller can test `if (status)` and index a table by code.  Nothing
+ *    is printed and no exception crosses the ABI.  Arguments are checked before
  *    anything is enqueued: an invalid argument enqueues nothing.  Errors found
  *    on the device (a negative position, a wait that timed out) set a device
  *    status word that swa_get_device_status() reads and clears.
  *  - Thread safety: calls are stateless apart from per-process caches: a
- *    driver entry point (set up once under a lock) and the launch register
- *    count of each attention-kernel variant (read once; every thread reads
- *    the same value).
+ *    driver entry point (set up once under a lock), the launch register
+ *    count of each attention-kernel variant (an atomic, read once; every
+ *    thread reads the same value) and the scratch address of
+ *    swa_attn_decode_ring_static (set up once per device under a lock).
  *  - The prefill / chunk / varlen kernels re-split their registers between
  *    warp groups and are written for 168 registers per thread at launch; a
  *    build that compiled them otherwise makes those calls return
@@ -89,7 +91,15 @@ SWA_API int swa_version(void);
  * their in-range coordinates.  Outputs (device memory, caller-allocated):
  *   classes: int8 [B, nqt, nkt] (may be NULL): 0 skip, 1 full, 2 partial;
  *   ranges:  int32 [B, nqt, 4]  (may be NULL): {live tiles, full tiles,
- *            first live tile, last live tile} (-1 when there is none);
+ *            first live tile, last live tile} (-1 when there is none).  In
+ *            mode 0 the live tiles of a query tile are always the contiguous
+ *            run first..last (the windows of consecutive rows overlap), and
+ *            the full tiles a contiguous run inside it, so the counts and the
+ *            ends locate both runs; in mode 1 the ring's physical order can
+ *            split the live tiles into two runs, on either side of the
+ *            slots that hold the oldest, invisible positions, which a single
+ *            [lo, hi) pair could not describe -- hence counts plus ends
+ *            rather than two half-open ranges;
  * with nqt = ceil(n_q / tile_q) and nkt = ceil(n_k / tile_k) (mode 0) or
  * ceil(W / tile_k) + ceil(n_q / tile_k) (mode 1).
  */
@@ -100,6 +110,9 @@ SWA_API int swa_block_meta(int key_mode, int B, int64_t n_q, int64_t n_k, const 
 /*
  * swa_attn_fwd -- tile-skipping prefill forward.
  * Passage: M003 note sections 03-04; Chapter 10 section 10.1.
+ * No metadata argument: the class of a (query tile, key tile) pair is a
+ * closed form of positions and W, which the kernel evaluates inline per tile
+ * (two integer compares), the same classification swa_block_meta writes out.
  *   q:   [B, H, N, d]    bf16, device     k, v: [B, Hkv, N, d] bf16, device
  *   out: [B, H, N, d]    bf16, device (written)
  *   lse: [B, H, N] fp32, device, or NULL: natural-log log-sum-exp of the
@@ -327,6 +340,11 @@ SWA_API int swa_attn_decode_ring_sink(const void *q, const void *k_ring, const v
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress with that device current) and caches it; make
  *    that first call before any stream capture.
+ *  - The cached address lives as long as the device's primary context: a
+ *    cudaDeviceReset() on that device (or anything else that destroys its
+ *    primary context) frees the array and leaves the cached address stale,
+ *    so a process that resets a device must not call this entry point on it
+ *    again.
  */
 SWA_API int swa_attn_decode_ring_static(const void *q, const void *k_ring, const void *v_ring,
                                         const int64_t *pos, void *out, float *lse, int B, int H,
@@ -341,6 +359,29 @@ SWA_API int swa_attn_decode_ring_static(const void *q, const void *k_ring, const
  */
 SWA_API int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,
                             void *stream);
+
+/*
+ * swa_selftest_wait -- runs the bounded device wait that every kernel of
+ * this library uses for failure detection, in a one-CTA kernel of its own
+ * (no copies, no tensor memory), so that the timeout path can be checked
+ * without breaking a real kernel.  The pages have no counterpart.
+ * Every mbarrier wait in the attention kernels gives up after a time limit,
+ * records SWA_ERR_TIMEOUT in the device status word and raises its CTA's
+ * abort flag; the CTA's other waits then give up at once, every role stops
+ * issuing work, copies and MMAs already issued are waited for, and the
+ * kernel returns instead of hanging the GPU.
+ *   limit_ns: 1000 .. 1000000000, the time limit of the first waiter.
+ *   arrive:   0: nobody arrives on the barriers: the first waiter gives up
+ *             after limit_ns, the 96 others follow through the abort flag,
+ *             and the next swa_get_device_status() returns SWA_ERR_TIMEOUT.
+ *             Nonzero: the barriers are arrived on before anyone waits, every
+ *             wait succeeds and the status word is left alone.
+ *   result:   int32 [5], device (written): result[w] for w = 0..3 counts the
+ *             lanes of warp w whose wait succeeded (warp 0 has one waiting
+ *             lane, warps 1-3 have 32 each); result[4] is the elapsed time
+ *             of the waits in microseconds.
+ */
+SWA_API int swa_selftest_wait(int64_t limit_ns, int arrive, int32_t *result, void *stream);
 
 /*
  * swa_get_device_status -- synchronise `stream`, then read and clear the

@@ -41,6 +41,7 @@ __all__ = [
     "swa_attn_decode_ring_sink",
     "swa_attn_decode_ring_static",
     "swa_ring_slot_positions",
+    "swa_selftest_wait",
     "swa_get_device_status",
     "swa_version",
     "swa_attn_fwd_seq_parallel",
@@ -355,6 +356,21 @@ def swa_ring_slot_positions(n_written, W: int, out=None):
     check("swa_ring_slot_positions", lib().swa_ring_slot_positions(
         B, _ptr(n_written), W, _ptr(out), _stream(n_written.device)))
     return out
+
+
+def swa_selftest_wait(limit_ns: int, arrive: bool = False, device=None):
+    """Run the library's bounded device wait in a one-CTA kernel of its own.
+
+    arrive=False: nobody arrives on the barrier, so the wait gives up after
+    limit_ns and swa_get_device_status() then reports SWA_ERR_TIMEOUT (5).
+    Returns int32 [5] on the device: lanes of warps 0..3 whose wait succeeded,
+    then the elapsed microseconds.
+    """
+    device = torch.device("cuda") if device is None else torch.device(device)
+    res = torch.zeros(5, dtype=torch.int32, device=device)
+    check("swa_selftest_wait", lib().swa_selftest_wait(int(limit_ns), 1 if arrive else 0,
+                                                       _ptr(res), _stream(device)))
+    return res
 
 
 def swa_get_device_status(stream=None) -> int:

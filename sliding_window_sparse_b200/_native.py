@@ -44,6 +44,7 @@ SIGNATURES = {
     "swa_attn_decode_ring": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i64, _f, _p, _sz, _p]),
     "swa_ring_slot_positions": (_i, [_i, _p, _i64, _p, _p]),
     "swa_attn_decode_ring_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i64, _f, _p]),
+    "swa_selftest_wait": (_i, [_i64, _i, _p, _p]),
     "swa_get_device_status": (_i, [_p]),
 }
 

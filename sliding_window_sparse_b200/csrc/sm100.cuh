@@ -7,6 +7,17 @@
 // gives up, records SWA_DEV_TIMEOUT in the device status word, raises the
 // CTA's abort flag and returns false; later waits in the CTA then return at
 // once, so a kernel with a broken handshake ends instead of hanging the GPU.
+//
+// What a kernel does after a wait returned false (its abort protocol):
+//  - a role that waited stops issuing: no further TMA copy, MMA or store;
+//  - warps whose lanes all wait take the decision together (mbar_wait_warp),
+//    so no warp-collective tcgen05 instruction runs with part of a warp;
+//  - before the CTA frees its tensor memory and exits, the TMA producer waits
+//    (mbar_drain, which ignores the abort flag but is bounded by the same
+//    limit) for every copy it issued to land in shared memory, and the MMA
+//    thread commits to a drain barrier and waits for every MMA it issued.
+//  The outputs of such a launch are invalid; swa_get_device_status() reports
+//  SWA_ERR_TIMEOUT.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -61,8 +72,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0u;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+// Bounded wait for the phase with the given parity to complete: false once
+// the CTA's abort flag is up or after limit_ns (then it raises the flag and
+// records SWA_DEV_TIMEOUT itself).
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
+                                                volatile int *abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
@@ -70,8 +84,34 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > SWA_WAIT_LIMIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
+      atomicOr(&g_swa_status, SWA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  return mbar_wait_limit(bar, parity, abort_flag, SWA_WAIT_LIMIT_NS);
+}
+// mbar_wait by every lane of a warp, with one outcome for the whole warp: a
+// lane that gave up makes the others give up too, so the warp stays converged
+// for the warp-collective instructions that follow.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int *abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag)) != 0;
+}
+// Teardown wait for work this thread issued itself (copies, MMAs): it does not
+// stop at the abort flag, since that work completes on its own; bounded all
+// the same (on expiry it records SWA_DEV_TIMEOUT and returns false).
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > SWA_WAIT_LIMIT_NS) {
       atomicOr(&g_swa_status, SWA_DEV_TIMEOUT);
       return false;
     }
@@ -219,32 +259,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x on the FMA pipe for a pair of values, x >= -125 (finite).
-// Range reduction x = n + f, n = round(x) (added to the exponent field),
-// f in [-1/2, 1/2]; 2^f from a degree-3 minimax polynomial for the relative
-// error (coefficients fitted by fit_exp2_poly.py: max relative error 7.5e-5).
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const float2 t = __fadd2_rn(x, magic);                      // n in the low mantissa bits
-  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-r.x, -r.y));
-  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                        make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// 2^x for two values at once on the MUFU: x packed to bf16 (round to nearest),
-// result as packed bf16 -- the form the P operand of the PV MMA takes.
-__device__ __forceinline__ uint32_t ex2_bf16x2(float lo, float hi) {
-  uint32_t x, y;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

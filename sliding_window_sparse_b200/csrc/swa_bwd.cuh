@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t BAR_EL = bar + 40;        // element-wise done with tile j (128 arrivals)
   const uint32_t BAR_DQF = bar + 48;       // dQ final
   const uint32_t BAR_DQE = bar + 56;       // dQ read out (128 arrivals)
+  const uint32_t BAR_DRAIN = bar + 64;     // the MMA thread's teardown
   const uint32_t BAR_KF = bar + 128;       // + 8 * stage
   const uint32_t BAR_KE = BAR_KF + 8 * NS;
   const uint32_t BAR_VF = BAR_KE + 8 * NS;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR_EL, 4 * 32);
     mbar_init(BAR_DQF, 1);
     mbar_init(BAR_DQE, 4 * 32);
+    mbar_init(BAR_DRAIN, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(BAR_KF + 8 * s, 1);
       mbar_init(BAR_KE + 8 * s, 1);
@@ -187,6 +189,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // --------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int q_iter = 0, kv_iter = 0;
+      bool k_ahead = false;  // K of iteration kv_iter issued, its V not (abort between them)
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         int b, h, t, k_lo;
         unit(u, b, h, t, k_lo);
@@ -209,8 +212,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sK + st * L::TILE + pn * (kBwdT * 128), &tm_k, BAR_KF + 8 * st, pn * 64,
                         kt * kBwdT, zk);
-          if (kv_iter >= NS && !mbar_wait(BAR_VE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag))
+          if (kv_iter >= NS &&
+              !mbar_wait(BAR_VE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag)) {
+            k_ahead = true;
             break;
+          }
           mbar_expect_tx(BAR_VF + 8 * st, L::TILE);
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
@@ -220,6 +226,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (*abort_flag) break;
       }
+      // every copy issued must land before the CTA ends
+      if (q_iter > 0) mbar_drain(BAR_QF, (q_iter - 1) & 1);
+      const int k_issued = kv_iter + (k_ahead ? 1 : 0);
+      for (int i = max(0, k_issued - NS); i < k_issued; ++i)
+        mbar_drain(BAR_KF + 8 * (i % NS), (i / NS) & 1);
+      for (int i = max(0, kv_iter - NS); i < kv_iter; ++i)
+        mbar_drain(BAR_VF + 8 * (i % NS), (i / NS) & 1);
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------- MMA issuer
@@ -305,6 +318,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_commit(BAR_DQF);
         ++q_iter;
       }
+      // every MMA issued must complete before the tensor memory is freed
+      tc_commit(BAR_DRAIN);
+      mbar_drain(BAR_DRAIN, 0);
     }
   } else {
     // --------------------------------------------------------------- element-wise
@@ -312,6 +328,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t s_cnt[2] = {0u, 0u}, dp_cnt = 0, u_iter = 0;
+    bool stop = false;  // a wait gave up (the whole warp): no more TMEM work or stores
     for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
       int b, h, t, k_lo;
       unit(u, b, h, t, k_lo);
@@ -345,7 +362,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int kt = k_lo + j;
         const int x = j & 1;
-        if (!mbar_wait(BAR_SF + 8 * x, s_cnt[x] & 1, abort_flag)) break;
+        if (!mbar_wait_warp(BAR_SF + 8 * x, s_cnt[x] & 1, abort_flag)) {
+          stop = true;
+          break;
+        }
         ++s_cnt[x];
         tc_fence_after();
         // allowed key columns of this row: positions in [qrow - W + 1, qrow] and < N
@@ -381,7 +401,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // phase 2: dS = P o (dP - D) as bf16 over the low half of this S buffer;
         // dP is released as soon as it is read
-        if (!mbar_wait(BAR_DPF, dp_cnt & 1, abort_flag)) break;
+        if (!mbar_wait_warp(BAR_DPF, dp_cnt & 1, abort_flag)) {
+          stop = true;
+          break;
+        }
         ++dp_cnt;
         tc_fence_after();
         auto dchunk = [&](int ch, const uint32_t (&dr)[32]) {
@@ -409,8 +432,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(BAR_EL);
       }
-      if (*abort_flag) break;
-      if (!mbar_wait(BAR_DQF, u_iter & 1, abort_flag)) break;
+      if (stop || __any_sync(0xffffffffu, *abort_flag)) break;
+      if (!mbar_wait_warp(BAR_DQF, u_iter & 1, abort_flag)) break;
       ++u_iter;
       tc_fence_after();
       {
@@ -459,6 +482,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t BAR_AE = bar + 48;        // dK, dV read out (128 arrivals)
   const uint32_t BAR_VEC = bar + 56;       // a step's lse2 / D columns staged (128 arrivals)
   const uint32_t BAR_DSF = bar + 64;       // dS^T of the step stored (128 arrivals)
+  const uint32_t BAR_DRAIN = bar + 72;     // the MMA thread's teardown
   const uint32_t BAR_QF = bar + 128;       // + 8 * stage
   const uint32_t BAR_QE = BAR_QF + 8 * NS;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
@@ -475,6 +499,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR_AE, 4 * 32);
     mbar_init(BAR_VEC, 4 * 32);
     mbar_init(BAR_DSF, 4 * 32);
+    mbar_init(BAR_DRAIN, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(BAR_QF + 8 * s, 1);
       mbar_init(BAR_QE + 8 * s, 1);
@@ -549,6 +574,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (*abort_flag) break;
       }
+      // every copy issued must land before the CTA ends
+      if (u_iter > 0) mbar_drain(BAR_KVF, (u_iter - 1) & 1);
+      for (int i = max(0, q_iter - NS); i < q_iter; ++i)
+        mbar_drain(BAR_QF + 8 * (i % NS), (i / NS) & 1);
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------- MMA issuer
@@ -624,6 +653,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_commit(BAR_AF);
         ++u_iter;
       }
+      // every MMA issued must complete before the tensor memory is freed
+      tc_commit(BAR_DRAIN);
+      mbar_drain(BAR_DRAIN, 0);
     }
   } else {
     // --------------------------------------------------------------- element-wise
@@ -663,8 +695,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int t = kt + s % nqt;
         if (s + 1 < n) col_vals(s + 1, l2n, ddn);  // loads in flight during this step
         const float *v2 = vec + (step & 1) * 2 * kBwdT;
-        if (!mbar_wait(BAR_VEC, step & 1, abort_flag) ||
-            !mbar_wait(BAR_SF, s_cnt & 1, abort_flag)) {
+        if (!mbar_wait_warp(BAR_VEC, step & 1, abort_flag) ||
+            !mbar_wait_warp(BAR_SF, s_cnt & 1, abort_flag)) {
           stop = true;
           break;
         }
@@ -711,7 +743,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(BAR_PF);
         // phase 2: dS^T = P^T o (dP^T - D), stored as bf16 over the low half of dP^T
-        if (!mbar_wait(BAR_DPF, s_cnt & 1, abort_flag)) {
+        if (!mbar_wait_warp(BAR_DPF, s_cnt & 1, abort_flag)) {
           stop = true;
           break;
         }
@@ -749,8 +781,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(BAR_DSF);
         if (s + 1 < n) stage(step + 1, l2n, ddn);
       }
-      if (stop || *abort_flag) break;
-      if (!mbar_wait(BAR_AF, u_iter & 1, abort_flag)) break;
+      if (stop || __any_sync(0xffffffffu, *abort_flag)) break;
+      if (!mbar_wait_warp(BAR_AF, u_iter & 1, abort_flag)) break;
       ++u_iter;
       tc_fence_after();
       // rows of this lane's 8-lane group: whole 128-byte segments per store

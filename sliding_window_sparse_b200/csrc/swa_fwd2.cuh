@@ -62,17 +62,6 @@ static_assert(4 * kRegsControl + 8 * kRegsSoftmax == (kFwd2Threads / 32) * kFwd2
 static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0 && kRegsSoftmax <= 256,
               "setmaxnreg counts are multiples of 8, at most 256");
 constexpr float kLazyRescaleLog2 = 8.0f;
-// The exponentials of the last kEmuCols columns of every tile are evaluated
-// on the FMA pipe (ex2_poly2) instead of the MUFU, to balance the two pipes.
-#ifndef SWA_EMU_COLS
-#define SWA_EMU_COLS 0
-#endif
-// Exponentials of P as packed bf16 pairs on the MUFU (ex2.approx.ftz.bf16x2).
-#ifndef SWA_EX2_BF16X2
-#define SWA_EX2_BF16X2 0
-#endif
-constexpr int kEmuCols = SWA_EMU_COLS;
-static_assert(kEmuCols % 16 == 0 && kEmuCols <= 128, "emulated columns in groups of 16");
 
 // MODE 0: linear [B, heads, N, D] layout.  MODE 1: chunk [B, heads, Tq, D] over
 // a ring [B, Hkv, W, D].  MODE 2: packed token-major [total, heads, D], sequence b
@@ -112,8 +101,8 @@ struct Fwd2Layout {
   static constexpr uint32_t OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + NV * KV_BYTES;
   // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
-  // o_full[2]
-  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 6;
+  // o_full[2], mma_drain
+  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 7;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t BYTES = OFF_MISC + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;
@@ -361,6 +350,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
   const uint32_t BAR_S = BAR_VE + 8 * NV;           // + 8 * tile
   const uint32_t BAR_P = BAR_S + 16;                // + 8 * tile
   const uint32_t BAR_O = BAR_P + 16;                // + 8 * tile
+  const uint32_t BAR_DRAIN = BAR_O + 16;            // the MMA thread's teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -381,6 +371,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
       mbar_init(BAR_P + 8 * x, 4 * 32);
       mbar_init(BAR_O + 8 * x, 1);
     }
+    mbar_init(BAR_DRAIN, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -449,6 +440,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int kv_iter = 0, q_iter = 0;
+      bool k_ahead = false;  // K of iteration kv_iter issued, its V not (abort between them)
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         Unit U = decode_unit(u, p);
         int64_t qs;
@@ -489,8 +481,11 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sK + sk * L::KV_BYTES + pn * (kKT * 128), mk, BAR_KF + 8 * sk, pn * 64,
                         MODE == 2 ? U.kvh : y0, MODE == 2 ? z + y0 : z);
-          if (kv_iter >= NV && !mbar_wait(BAR_VE + 8 * sv, ((kv_iter / NV) - 1) & 1, abort_flag))
+          if (kv_iter >= NV &&
+              !mbar_wait(BAR_VE + 8 * sv, ((kv_iter / NV) - 1) & 1, abort_flag)) {
+            k_ahead = true;
             break;
+          }
           mbar_expect_tx(BAR_VF + 8 * sv, L::KV_BYTES);
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
@@ -500,6 +495,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         }
         if (*abort_flag) break;
       }
+      // every copy issued must land before the CTA ends: wait for the last
+      // phase of each barrier that a copy was issued on
+      if (q_iter > 0) mbar_drain(BAR_QF, (q_iter - 1) & 1);
+      const int k_issued = kv_iter + (k_ahead ? 1 : 0);
+      for (int i = max(0, k_issued - NK); i < k_issued; ++i)
+        mbar_drain(BAR_KF + 8 * (i % NK), (i / NK) & 1);
+      for (int i = max(0, kv_iter - NV); i < kv_iter; ++i)
+        mbar_drain(BAR_VF + 8 * (i % NV), (i / NV) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -532,7 +535,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         int64_t qs;
         int len;
         if (unit_start(U, qs, len)) continue;
-        mbar_wait(BAR_QF, q_iter & 1, abort_flag);
+        if (!mbar_wait(BAR_QF, q_iter & 1, abort_flag)) break;
         tc_fence_after();
         Walker2<MODE, SINK> wk;
         wk.init(U, p, qs, len);
@@ -547,7 +550,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         bool has_next = wk.next_live(k, src, y0, na, nb);
         {
           const int sk = kv_iter % NK;
-          mbar_wait(BAR_KF + 8 * sk, (kv_iter / NK) & 1, abort_flag);
+          if (!mbar_wait(BAR_KF + 8 * sk, (kv_iter / NK) & 1, abort_flag)) break;
           tc_fence_after();
           if (ca) issue_s(0, sk);
           if (cb) issue_s(1, sk);
@@ -557,7 +560,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         bool b_ahead = false;
         if (MODE != 1 && has_next && nb && !cb) {
           const int sk1 = (kv_iter + 1) % NK;
-          mbar_wait(BAR_KF + 8 * sk1, ((kv_iter + 1) / NK) & 1, abort_flag);
+          if (!mbar_wait(BAR_KF + 8 * sk1, ((kv_iter + 1) / NK) & 1, abort_flag)) break;
           tc_fence_after();
           issue_s(1, sk1);
           b_ahead = true;
@@ -565,13 +568,20 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         tc_commit(BAR_KE + 8 * (kv_iter % NK));  // K(first) is read by both S MMAs
         bool o_done[2] = {false, false};
         const bool b_contig = MODE != 1 && (!SINK || p.n_sink == 0 || p.pair_heads);
+        bool stop = false;  // a wait gave up: issue nothing more
         while (have) {
           if (!has_next) tc_commit(BAR_QE);  // every S of this unit is issued
           const int sv = kv_iter % NV;
           const int skn = (kv_iter + 1) % NK;
-          mbar_wait(BAR_VF + 8 * sv, (kv_iter / NV) & 1, abort_flag);
+          if (!mbar_wait(BAR_VF + 8 * sv, (kv_iter / NV) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
           if (ca) {
-            mbar_wait(BAR_P, p_cnt[0] & 1, abort_flag);
+            if (!mbar_wait(BAR_P, p_cnt[0] & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
             ++p_cnt[0];
             tc_fence_after();
             issue_pv(0, sv, !first[0]);
@@ -584,12 +594,18 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             }
           }
           if (has_next) {
-            mbar_wait(BAR_KF + 8 * skn, ((kv_iter + 1) / NK) & 1, abort_flag);
+            if (!mbar_wait(BAR_KF + 8 * skn, ((kv_iter + 1) / NK) & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
             tc_fence_after();
             if (na) issue_s(0, skn);
           }
           if (cb) {
-            mbar_wait(BAR_P + 8, p_cnt[1] & 1, abort_flag);
+            if (!mbar_wait(BAR_P + 8, p_cnt[1] & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
             ++p_cnt[1];
             tc_fence_after();
             issue_pv(1, sv, !first[1]);
@@ -611,6 +627,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           have = has_next;
           if (have) has_next = wk.next_live(k, src, y0, na, nb);
         }
+        if (stop) break;
         // o_final completes once per unit in which the tile had work; its next
         // completion needs that tile's softmax to hand over its next P, so it
         // can never run two phases ahead of the waiting softmax warps
@@ -618,6 +635,9 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         if (!first[1] && !o_done[1]) tc_commit(BAR_O + 8);
         ++q_iter;
       }
+      // every MMA issued must complete before the tensor memory is freed
+      tc_commit(BAR_DRAIN);
+      mbar_drain(BAR_DRAIN, 0);
     }
   }  // warps 2 and 3 have no role
   } else {
@@ -630,6 +650,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     const uint32_t tS = tmem + x * 128 + lane_off;
     const uint32_t tO = tmem + 256 + x * D + lane_off;
     uint32_t s_cnt = 0, u_iter = 0;
+    bool stop = false;  // a wait gave up (the whole warp): no more TMEM work or stores
     for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
       Unit U = decode_unit(u, p);
       int64_t qs;
@@ -645,7 +666,10 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
       while (wk.next(k, src, y0, ca, cb)) {
         const int cls = x == 0 ? ca : cb;
         if (!cls) continue;
-        mbar_wait(BAR_S + 8 * x, s_cnt & 1, abort_flag);
+        if (!mbar_wait_warp(BAR_S + 8 * x, s_cnt & 1, abort_flag)) {
+          stop = true;
+          break;
+        }
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[128];
@@ -701,42 +725,9 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         float2 *s2 = reinterpret_cast<float2 *>(s);
 #pragma unroll
         for (int c = 0; c < kKT / 2; ++c) s2[c] = __ffma2_rn(s2[c], sc2, nm2);
-#if SWA_EX2_BF16X2
-        // P = 2^x evaluated two columns per MUFU op directly in bf16 (the PV MMA's
-        // operand type); the row sum adds exactly those bf16 weights
-        uint32_t pk[kKT / 2];
+        // exponentials on the MUFU (a masked column gives 2^-inf = 0)
 #pragma unroll
-        for (int c = 0; c < kKT / 2; ++c) pk[c] = ex2_bf16x2(s2[c].x, s2[c].y);
-        float2 sm2[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kKT / 2; c += 4)
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            sm2[i] = __fadd2_rn(sm2[i], make_float2(__uint_as_float(pk[c + i] << 16),
-                                                    __uint_as_float(pk[c + i] & 0xFFFF0000u)));
-        const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
-        const float rs = sa.x + sa.y;
-        l_run = l_run * alpha + rs;
-        m_run = m_new;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t half[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) half[i] = pk[h2 * 32 + i];
-          tmem_st32(tS + h2 * 32, half);
-        }
-#else
-        // exponentials: MUFU for the first columns, FMA-pipe polynomial for the last
-        // kEmuCols (a masked column clamps to 2^-125 there, which is numerically 0
-        // next to the row maximum's 2^0 and is cleared with O and l by any later
-        // rescale)
-#pragma unroll
-        for (int c = 0; c < kKT - kEmuCols; ++c) s[c] = ex2(s[c]);
-#pragma unroll
-        for (int c = (kKT - kEmuCols) / 2; c < kKT / 2; ++c)
-          s2[c] = ex2_poly2(make_float2(fmaxf(s2[c].x, -125.f), fmaxf(s2[c].y, -125.f)));
+        for (int c = 0; c < kKT; ++c) s[c] = ex2(s[c]);
         float2 sm2[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
@@ -756,7 +747,6 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
           for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[h2 * 64 + 2 * i], s[h2 * 64 + 2 * i + 1]);
           tmem_st32(tS + h2 * 32, pk);
         }
-#endif
         // O_X is stable: PV_X of the previous tile was issued before this S_X
         if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -774,9 +764,10 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         mbar_arrive(BAR_P + 8 * x);
         ++nt;
       }
+      if (stop) break;
       if (nt > 0) {
         // every PV of this unit is done
-        mbar_wait(BAR_O + 8 * x, u_iter & 1, abort_flag);
+        if (!mbar_wait_warp(BAR_O + 8 * x, u_iter & 1, abort_flag)) break;
         ++u_iter;
         tc_fence_after();
         const float inv_l = 1.f / l_run;

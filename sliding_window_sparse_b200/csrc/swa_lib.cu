@@ -10,6 +10,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -19,6 +20,7 @@
 #include "swa_decode.cuh"
 #include "swa_fwd2.cuh"
 #include "swa_meta.cuh"
+#include "swa_selftest.cuh"
 #include "swa_tile.cuh"
 
 namespace {
@@ -111,13 +113,17 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
     return SWA_ERR_CUDA;
   // The kernel's warpgroups re-split the registers it is launched with
   // (setmaxnreg); that split assumes exactly kFwd2LaunchRegs per thread.
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
+  // The count is read once per kernel variant; concurrent first calls may
+  // both read it and store the same value.
+  static std::atomic<int> launch_regs{-1};
+  int regs = launch_regs.load(std::memory_order_relaxed);
+  if (regs < 0) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SWA_ERR_CUDA;
-    launch_regs = fa.numRegs;
+    regs = fa.numRegs;
+    launch_regs.store(regs, std::memory_order_relaxed);
   }
-  if (launch_regs != swa::kFwd2LaunchRegs) return SWA_ERR_UNSUPPORTED;
+  if (regs != swa::kFwd2LaunchRegs) return SWA_ERR_UNSUPPORTED;
   p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
   const int64_t units = p.pair_heads
                             ? static_cast<int64_t>(p.B) * p.Hkv * (p.G / 2) * p.nqt
@@ -586,6 +592,13 @@ int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t 
   return check_launch();
 }
 
+int swa_selftest_wait(int64_t limit_ns, int arrive, int32_t *result, void *stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000 || !result) return SWA_ERR_INVALID_ARG;
+  swa::selftest_wait_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ns), arrive ? 1 : 0, result);
+  return check_launch();
+}
+
 int swa_get_device_status(void *stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SWA_ERR_CUDA;
   unsigned int v = 0, zero = 0;
@@ -622,7 +635,9 @@ int swa_get_device_status(void *stream) {
 // Host code cannot use the array's name as a device address, so the first
 // call on each device looks the address up with cudaGetSymbolAddress while
 // that device is current and caches it; make that first call before any
-// stream capture.
+// stream capture.  The cached address is valid for the life of the device's
+// primary context: after a cudaDeviceReset() of that device it is stale, and
+// this entry point must not be called on that device again.
 // ---------------------------------------------------------------------------
 namespace {
 

@@ -82,11 +82,16 @@ def test_workload_sampled_rows(swa, name):
     w = WORKLOADS[name]
     q, k, v = prefill_inputs(w)
     out = _run(swa, q, k, v, w.W, w.scale)
+    # the first and last row of every query tile, and the rows around the window
+    # edge (W - 2 .. W) and the last row, each at a random (b, h); sample_rows
+    # keeps every listed row
     edges = []
     for t in range(0, w.N, 128):
         edges += [t, t + 127]
     edges += [w.W - 2, w.W - 1, w.W, w.N - 1]
-    rows = sample_rows(w.B, w.H, w.N, 384, seed=7, extra=edges[:128])
+    rows = sample_rows(w.B, w.H, w.N, 384, seed=7, extra=edges)
+    listed = set(int(i) for i in rows[:, 2])
+    assert all(i in listed for i in edges)
     ref = oracle.swa_forward(q, k, v, w.W, w.scale, rows=rows)
     got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_close(got, ref, what=name)
