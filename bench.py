@@ -85,6 +85,10 @@ def useful_flops(w) -> int:
         from swa_inputs.workloads import seq_lens
 
         return 4 * w.d * w.H * sum(sequence_pairs(int(n), w.W, w.n_sink) for n in seq_lens(w))
+    if w.kind == "varlen_backward":
+        from swa_inputs.workloads import seq_lens
+
+        return 10 * w.d * w.H * sum(sequence_pairs(int(n), w.W, w.n_sink) for n in seq_lens(w))
     if w.kind == "chunk":
         pairs = sum(valid_pairs_row(w.q_start + t, w.W) +
                     min(w.n_sink, max(0, w.q_start + t - w.W + 1))
@@ -121,6 +125,11 @@ def algorithmic_bytes(w) -> int:
 
         total = int(cu_seqlens(w)[-1])
         return e * w.d * (2 * w.H * total + 2 * w.Hkv * total)
+    if w.kind == "varlen_backward":
+        from swa_inputs.workloads import cu_seqlens
+
+        total = int(cu_seqlens(w)[-1])
+        return e * w.d * (4 * w.H * total + 4 * w.Hkv * total) + 4 * w.H * total
     if w.kind == "chunk":
         rows = sum(chunk_rows(w))
         return e * w.d * (2 * w.H * rows + 2 * w.Hkv * (rows + w.B * w.W))
@@ -157,7 +166,7 @@ def describe(w) -> str:
     sink = f" sinks{w.n_sink}" if w.n_sink else ""
     if w.kind in ("prefill", "backward"):
         return f"{w.name}: B{w.B} H{w.H} Hkv{w.Hkv} N{w.N} d{w.d} W{w.W}{sink}"
-    if w.kind == "varlen":
+    if w.kind in ("varlen", "varlen_backward"):
         return (f"{w.name}: {w.n_seq} packed sequences, lengths U[{w.len_lo},{w.len_hi}], "
                 f"H{w.H} Hkv{w.Hkv} d{w.d} W{w.W}{sink}")
     if w.kind == "chunk":
@@ -286,14 +295,23 @@ def make_inputs(w, device, seed_offset=0):
         x["out"], x["lse"] = swa.swa_attn_fwd(x["q"], x["k"], x["v"], w.W, w.scale,
                                               return_lse=True)
         return x
-    if w.kind == "varlen":
-        from swa_inputs.workloads import cu_seqlens
+    if w.kind in ("varlen", "varlen_backward"):
+        from swa_inputs.workloads import cu_seqlens, seq_lens
 
         cu = cu_seqlens(w)
         total = int(cu[-1])
-        return {"q": g("q", (total, w.H, w.d)), "k": g("k", (total, w.Hkv, w.d)),
-                "v": g("v", (total, w.Hkv, w.d)),
-                "cu_seqlens": torch.tensor(cu, dtype=torch.int64, device=device)}
+        x = {"q": g("q", (total, w.H, w.d)), "k": g("k", (total, w.Hkv, w.d)),
+             "v": g("v", (total, w.Hkv, w.d)),
+             "cu_seqlens": torch.tensor(cu, dtype=torch.int64, device=device)}
+        if w.kind == "varlen_backward":
+            import sliding_window_sparse_b200 as swa
+
+            x["dout"] = g("extra", (total, w.H, w.d))
+            # the forward's output and LSE are inputs of the backward (made once, untimed)
+            x["out"], x["lse"] = swa.swa_attn_varlen(x["q"], x["k"], x["v"], x["cu_seqlens"],
+                                                     int(max(seq_lens(w))), w.W, w.scale,
+                                                     n_sink=w.n_sink, return_lse=True)
+        return x
     if w.kind == "chunk":
         x = {"q": g("q", (w.B, w.H, w.Tq, w.d)),
              "k_new": g("k_new", (w.B, w.Hkv, w.Tq, w.d)),
@@ -333,6 +351,18 @@ def make_call(w, x, swa):
                          dtype=torch.uint8, device=x["q"].device)
         return (lambda: swa.swa_attn_bwd(x["q"], x["k"], x["v"], x["out"], x["dout"], x["lse"],
                                          w.W, w.scale, dq=dq, dk=dk, dv=dv, workspace=ws), dq, 2)
+    if w.kind == "varlen_backward":
+        from swa_inputs.workloads import seq_lens
+
+        dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+        total = x["q"].shape[0]
+        ws = torch.empty(int(swa.lib().swa_attn_varlen_bwd_workspace_bytes(w.H, total)),
+                         dtype=torch.uint8, device=x["q"].device)
+        max_len = int(max(seq_lens(w)))
+        return (lambda: swa.swa_attn_varlen_bwd(x["q"], x["k"], x["v"], x["cu_seqlens"], max_len,
+                                                x["out"], x["dout"], x["lse"], w.W, w.scale,
+                                                n_sink=w.n_sink, dq=dq, dk=dk, dv=dv,
+                                                workspace=ws), dq, 2)
     if w.kind == "varlen":
         from swa_inputs.workloads import seq_lens
 
@@ -605,7 +635,8 @@ def run_native(args):
     if not args.headline_only:
         for name in ("mistral_prefill", "narrow_window", "chunk_ring", "decode_ring",
                      "varlen_prefill", "mistral_prefill_sink", "chunk_ring_ragged",
-                     "decode_ring_sink", "chunk_ring_sink", "mistral_backward"):
+                     "decode_ring_sink", "chunk_ring_sink", "mistral_backward",
+                     "varlen_backward"):
             if name == headline:
                 continue
             pw = WORKLOADS[name]
@@ -631,7 +662,8 @@ def run_native(args):
                                            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                            "frac": tf / peaks["bf16_tflops"],
                                            "traffic": (profiled_traffic("fwd2_kernel", name)
-                                                       if pw.kind != "backward" else None)}})
+                                                       if "backward" not in pw.kind
+                                                       else None)}})
             if (rank == 0 and world == 1 and not args.no_cpu_baseline
                     and name in CPU_BASELINE_PATHS):
                 entry["cpu_baseline"] = cpu_baseline(pw, host_inputs_of(pw, px),

@@ -195,6 +195,51 @@ SWA_API int swa_attn_bwd(const void *q, const void *k, const void *v, const void
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * swa_attn_bwd_sink -- gradients of swa_attn_fwd_sink (attention sinks).
+ * Passage: M003 note sections 07-08 (gradients under the same mask as the
+ * outputs); sparse-attention taxonomy page section 3.2 for the mask: query i
+ * reads key j iff j <= i and (j >= i - W + 1 or j < n_sink).  Key tile 0,
+ * which holds the sinks, is read by every query tile.
+ *   n_sink: 0 <= n_sink <= 128 (0 is swa_attn_bwd); lse: from
+ *   swa_attn_fwd_sink with the same n_sink.
+ * Other arguments, layouts, workspace and limits as swa_attn_bwd.
+ */
+SWA_API int swa_attn_bwd_sink(const void *q, const void *k, const void *v, const void *out,
+                              const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                              int B, int H, int Hkv, int64_t N, int d, int64_t W, int n_sink,
+                              float scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * swa_attn_varlen_bwd_workspace_bytes -- bytes of scratch swa_attn_varlen_bwd
+ * needs: one fp32 D_i per (head, token): H * total * 4, 256-aligned.
+ */
+SWA_API size_t swa_attn_varlen_bwd_workspace_bytes(int H, int64_t total);
+
+/*
+ * swa_attn_varlen_bwd -- gradients of swa_attn_varlen (packed sequences, each
+ * with its own window, optional sinks).
+ * Passage: M003 note sections 07-08; "Dense attention vs sparse SWA" blog
+ * section 5.2 tip 4 (windows per sequence, no leakage across cu_seqlens);
+ * taxonomy page section 3.2 for the sinks.  Same gradients as swa_attn_bwd,
+ * per sequence; nothing flows between sequences.
+ *   q, out, dout, dq: [total, H, d] bf16, device (token-major, as the forward)
+ *   k, v, dk, dv:     [total, Hkv, d] bf16, device
+ *   cu_seqlens: int64 [n_seq + 1], device, as swa_attn_varlen (bad offsets
+ *        set SWA_ERR_DEVICE and the sequence is skipped).
+ *   lse: [H, total] fp32, device: the forward's natural-log LSE.
+ *   n_sink: 0 <= n_sink <= 128, as in the forward.
+ *   workspace: at least swa_attn_varlen_bwd_workspace_bytes(H, total) bytes.
+ * Rows of tokens outside every sequence of dq, dk, dv are not written.
+ * Limits as swa_attn_varlen.
+ */
+SWA_API int swa_attn_varlen_bwd(const void *q, const void *k, const void *v,
+                                const int64_t *cu_seqlens, const void *out, const void *dout,
+                                const float *lse, void *dq, void *dk, void *dv, int n_seq,
+                                int64_t total, int64_t max_seqlen, int H, int Hkv, int d,
+                                int64_t W, int n_sink, float scale, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * swa_attn_chunk_ring -- chunked prefill over a W-slot ring-buffer KV cache.
  * Passage: Chapter 10 section 10.2 (a chunk of T_q queries needs the union of
  * W + T_q - 1 keys; the persistent cache keeps only the last W); M003 note

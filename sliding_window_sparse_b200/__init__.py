@@ -31,6 +31,7 @@ __all__ = [
     "swa_attn_fwd",
     "swa_attn_fwd_sink",
     "swa_attn_bwd",
+    "swa_attn_varlen_bwd",
     "swa_attn_varlen",
     "swa_attn_chunk_ring",
     "swa_attn_chunk_ring_ragged",
@@ -131,10 +132,11 @@ def swa_attn_fwd(q, k, v, W: int, scale: float | None = None, out=None, lse=None
 
 
 def swa_attn_bwd(q, k, v, out, dout, lse, W: int, scale: float | None = None, dq=None, dk=None,
-                 dv=None, workspace=None):
+                 dv=None, workspace=None, n_sink: int = 0):
     """Gradients of swa_attn_fwd: returns (dq [B,H,N,d], dk, dv [B,Hkv,N,d]).
 
     out and lse are the forward's output and natural-log LSE; dout is the incoming gradient.
+    n_sink > 0: gradients of swa_attn_fwd_sink with the same sinks (swa_attn_bwd_sink).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _need(t, n, dims=4)
@@ -153,11 +155,53 @@ def swa_attn_bwd(q, k, v, out, dout, lse, W: int, scale: float | None = None, dq
     need = int(lib().swa_attn_bwd_workspace_bytes(B, H, N))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    check("swa_attn_bwd",
-          lib().swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
-                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d, W, scale,
-                             _ptr(workspace), workspace.numel() * workspace.element_size(),
-                             _stream(q.device)))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if n_sink:
+        check("swa_attn_bwd_sink",
+              lib().swa_attn_bwd_sink(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d, W, n_sink,
+                                      scale, _ptr(workspace), ws_bytes, _stream(q.device)))
+    else:
+        check("swa_attn_bwd",
+              lib().swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d, W, scale,
+                                 _ptr(workspace), ws_bytes, _stream(q.device)))
+    return dq, dk, dv
+
+
+def swa_attn_varlen_bwd(q, k, v, cu_seqlens, max_seqlen: int, out, dout, lse, W: int,
+                        scale: float | None = None, n_sink: int = 0, dq=None, dk=None, dv=None,
+                        workspace=None):
+    """Gradients of swa_attn_varlen: returns (dq [total,H,d], dk, dv [total,Hkv,d]).
+
+    out and lse ([H, total]) are the forward's; dout is the incoming gradient.  Rows of
+    tokens outside every sequence keep what dq / dk / dv held (zeros when allocated here).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, dims=3)
+    _need(cu_seqlens, "cu_seqlens", torch.int64, 1)
+    _need(lse, "lse", torch.float32, 2)
+    total, H, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (total, Hkv, d) or tuple(v.shape) != (total, Hkv, d):
+        raise ValueError("k and v must be [total, Hkv, d] matching q")
+    if tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("out and dout must match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.zeros_like(q) if dq is None else dq
+    dk = torch.zeros_like(k) if dk is None else dk
+    dv = torch.zeros_like(v) if dv is None else dv
+    need = int(lib().swa_attn_varlen_bwd_workspace_bytes(H, total))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check("swa_attn_varlen_bwd",
+          lib().swa_attn_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out),
+                                    _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                                    cu_seqlens.shape[0] - 1, total, max_seqlen, H, Hkv, d, W,
+                                    n_sink, scale, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    _stream(q.device)))
     return dq, dk, dv
 
 

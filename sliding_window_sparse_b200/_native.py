@@ -35,6 +35,11 @@ SIGNATURES = {
     "swa_attn_bwd_workspace_bytes": (_sz, [_i, _i, _i64]),
     "swa_attn_bwd": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i64, _i, _i64, _f, _p,
                           _sz, _p]),
+    "swa_attn_bwd_sink": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i64, _i, _i64, _i,
+                               _f, _p, _sz, _p]),
+    "swa_attn_varlen_bwd_workspace_bytes": (_sz, [_i, _i64]),
+    "swa_attn_varlen_bwd": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i64, _i, _i,
+                                 _i, _i64, _i, _f, _p, _sz, _p]),
     "swa_attn_chunk_ring_sink": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i64,
                                       _i, _i64, _f, _i, _p]),
     "swa_attn_chunk_ring_ragged": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i64, _i,

@@ -25,6 +25,14 @@
 // Key tile j and query tile t interact iff some key of j is in the window of
 // some query of t (the M003 note, section 04's skip rule); partial tiles are
 // masked per row with 128-bit column masks.
+//
+// Layouts (MODE): 0 = [B, heads, N, D] per tensor; 2 = packed token-major
+// [total, heads, D] with sequence b on tokens cu_seqlens[b] .. cu_seqlens[b+1]-1
+// and positions restarting at 0 in each sequence (the "Dense attention vs
+// sparse SWA" blog, section 5.2 tip 4: the window is per sequence).  SINK adds
+// attention sinks (sparse-attention taxonomy page, section 3.2): key j < n_sink
+// stays visible to every later query of its sequence, so query tile t also
+// reads key tile 0, and key tile 0 is read by every query tile.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -37,6 +45,7 @@ namespace swa {
 constexpr int kBwdT = 128;            // query and key tile rows
 constexpr int kBwdThreads = 6 * 32;   // producer, MMA issuer, 4 element-wise warps
 
+// MODE 2: out, dout, dq [total, H, D]; dk, dv [total, Hkv, D]; lse, delta [H, total].
 struct BwdParams {
   const __nv_bfloat16 *out;   // [B, H, N, D]
   const __nv_bfloat16 *dout;  // [B, H, N, D]
@@ -45,11 +54,14 @@ struct BwdParams {
   __nv_bfloat16 *dq;          // [B, H, N, D]
   __nv_bfloat16 *dk, *dv;     // [B, Hkv, N, D]
   int B = 0, H = 0, Hkv = 0, G = 0;
-  int N = 0;
+  int N = 0;                  // MODE 2: the longest sequence
   int W = 0;                  // window, clamped to N + kBwdT
   float scale = 0.f, scale_log2 = 0.f;
   int nt = 0;                 // tiles per (b, head): ceil(N / 128)
   int n_units = 0;
+  const int64_t *cu_seqlens = nullptr;  // MODE 2: [B + 1]
+  int64_t total = 0;                    // MODE 2: packed tokens
+  int n_sink = 0;                       // SINK: keys 0 .. n_sink-1 of each sequence
 };
 
 template <int D>
@@ -104,9 +116,56 @@ __device__ __forceinline__ void col_mask(int lo, int hi, uint32_t (&mw)[4]) {
   for (int w = 0; w < 4; ++w) mw[w] = range_bits(lo - 32 * w, hi - 32 * w);
 }
 
+// The sequence of batch entry b: its first token `a` (MODE 2; 0 otherwise) and
+// its length.  Returns 1 when MODE 2 offsets are out of range.
+template <int MODE>
+__device__ __forceinline__ int bwd_seq(const BwdParams &p, int b, int64_t &a, int &len) {
+  a = 0;
+  len = p.N;
+  if (MODE == 2) {
+    const int64_t s = p.cu_seqlens[b], e = p.cu_seqlens[b + 1];
+    if (s < 0 || e < s || e - s > p.N || e > p.total) return 1;
+    a = s;
+    len = static_cast<int>(e - s);
+  }
+  return 0;
+}
+
+// The key tiles of query tile t in the dQ kernel's order: key tile 0 first
+// when it holds sinks the window does not reach, then k_lo .. t.
+struct DqTiles {
+  int k_lo, n;
+  bool sink;
+  __device__ __forceinline__ int kt(int j) const {
+    return sink ? (j == 0 ? 0 : k_lo + j - 1) : k_lo + j;
+  }
+};
+template <bool SINK>
+__device__ __forceinline__ DqTiles dq_tiles(const BwdParams &p, int t) {
+  DqTiles r;
+  r.k_lo = max(t * kBwdT - (p.W - 1), 0) / kBwdT;
+  r.sink = SINK && p.n_sink > 0 && r.k_lo > 0;
+  r.n = t - r.k_lo + 1 + (r.sink ? 1 : 0);
+  return r;
+}
+
+// Element offset of (row r of head h) in a [B, heads, N, D] tensor (MODE 0,
+// b = batch entry, r from 0) or a [total, heads, D] one (MODE 2, token a + r).
+template <int MODE>
+__device__ __forceinline__ int64_t bwd_row(const BwdParams &p, int b, int64_t a, int heads, int h,
+                                           int r) {
+  return MODE == 2 ? (a + r) * heads + h : (static_cast<int64_t>(b) * heads + h) * p.N + r;
+}
+// Index of (row r, head h) in the per-row fp32 arrays lse and delta.
+template <int MODE>
+__device__ __forceinline__ int64_t bwd_vec(const BwdParams &p, int b, int64_t a, int h, int r) {
+  return MODE == 2 ? static_cast<int64_t>(h) * p.total + a + r
+                   : (static_cast<int64_t>(b) * p.H + h) * p.N + r;
+}
+
 // ---------------------------------------------------------------------------------- dQ
 // Unit u: (b, h, query tile t), heaviest tiles first.
-template <int D>
+template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v,
@@ -171,14 +230,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // tensor memory: S double buffer [0, 256), dP [256, 384), dQ [384, 384 + D)
   const uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
 
-  // unit -> (b, h, t); the key tiles of query tile t are [k_lo, t]
-  auto unit = [&](int u, int &b, int &h, int &t, int &k_lo) {
+  // unit -> (b, h, t) and its sequence; 0: run it, 1: bad sequence offsets
+  // (skip, flag), 2: the query tile lies past the sequence's end (skip).
+  // Every role evaluates it identically, so they skip the same units.
+  auto unit = [&](int u, int &b, int &h, int &t, int64_t &a, int &len) -> int {
     const int per_t = p.B * p.H;
     t = p.nt - 1 - u / per_t;
     const int bh = u % per_t;
     b = bh / p.H;
     h = bh % p.H;
-    k_lo = max(t * kBwdT - (p.W - 1), 0) / kBwdT;
+    if (bwd_seq<MODE>(p, b, a, len)) return 1;
+    return t * kBwdT >= len ? 2 : 0;
   };
   auto unit_of = [&](int i) -> int {
     const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
@@ -191,19 +253,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int q_iter = 0, kv_iter = 0;
       bool k_ahead = false;  // K of iteration kv_iter issued, its V not (abort between them)
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        int b, h, t, k_lo;
-        unit(u, b, h, t, k_lo);
+        int b, h, t, len;
+        int64_t a;
+        const int ust = unit(u, b, h, t, a, len);
+        if (ust) {
+          if (ust == 1) atomicOr(&g_swa_status, SWA_DEV_BADARG);
+          continue;
+        }
+        const DqTiles tl = dq_tiles<SINK>(p, t);
         if (q_iter > 0 && !mbar_wait(BAR_QE, (q_iter - 1) & 1, abort_flag)) break;
         mbar_expect_tx(BAR_QF, 2 * L::TILE);
-        const int zq = b * p.H + h;
+        // MODE 2 maps are {D, heads, tokens}: (head, token) replace (row, plane)
+        const int qy = MODE == 2 ? h : t * kBwdT;
+        const int qz = MODE == 2 ? static_cast<int>(a) + t * kBwdT : b * p.H + h;
 #pragma unroll
         for (int pn = 0; pn < L::PANELS; ++pn) {
-          tma_load_3d(sQ + pn * (kBwdT * 128), &tm_q, BAR_QF, pn * 64, t * kBwdT, zq);
-          tma_load_3d(sDO + pn * (kBwdT * 128), &tm_do, BAR_QF, pn * 64, t * kBwdT, zq);
+          tma_load_3d(sQ + pn * (kBwdT * 128), &tm_q, BAR_QF, pn * 64, qy, qz);
+          tma_load_3d(sDO + pn * (kBwdT * 128), &tm_do, BAR_QF, pn * 64, qy, qz);
         }
         ++q_iter;
-        const int zk = b * p.Hkv + h / p.G;
-        for (int kt = k_lo; kt <= t; ++kt) {
+        for (int j = 0; j < tl.n; ++j) {
+          const int kt = tl.kt(j);
+          const int ky = MODE == 2 ? h / p.G : kt * kBwdT;
+          const int kz = MODE == 2 ? static_cast<int>(a) + kt * kBwdT : b * p.Hkv + h / p.G;
           const int st = kv_iter % NS;
           if (kv_iter >= NS && !mbar_wait(BAR_KE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag))
             break;
@@ -211,7 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sK + st * L::TILE + pn * (kBwdT * 128), &tm_k, BAR_KF + 8 * st, pn * 64,
-                        kt * kBwdT, zk);
+                        ky, kz);
           if (kv_iter >= NS &&
               !mbar_wait(BAR_VE + 8 * st, ((kv_iter / NS) - 1) & 1, abort_flag)) {
             k_ahead = true;
@@ -221,7 +293,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_3d(sV + st * L::TILE + pn * (kBwdT * 128), &tm_v, BAR_VF + 8 * st, pn * 64,
-                        kt * kBwdT, zk);
+                        ky, kz);
           ++kv_iter;
         }
         if (*abort_flag) break;
@@ -251,9 +323,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        int b, h, t, k_lo;
-        unit(u, b, h, t, k_lo);
-        const int n = t - k_lo + 1;
+        int b, h, t, len;
+        int64_t a;
+        if (unit(u, b, h, t, a, len)) continue;
+        const int n = dq_tiles<SINK>(p, t).n;
         if (!mbar_wait(BAR_QF, q_iter & 1, abort_flag)) break;
         tc_fence_after();
         const int kv0 = kv_iter;
@@ -330,15 +403,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t s_cnt[2] = {0u, 0u}, dp_cnt = 0, u_iter = 0;
     bool stop = false;  // a wait gave up (the whole warp): no more TMEM work or stores
     for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-      int b, h, t, k_lo;
-      unit(u, b, h, t, k_lo);
-      const int n = t - k_lo + 1;
+      int b, h, t, len;
+      int64_t a;
+      if (unit(u, b, h, t, a, len)) continue;
+      const DqTiles tl = dq_tiles<SINK>(p, t);
+      const int n = tl.n;
       const int qrow = t * kBwdT + row;
-      const bool valid = qrow < p.N;
-      const int64_t r = (static_cast<int64_t>(b) * p.H + h) * p.N + qrow;
+      const bool valid = qrow < len;
       // D_i = <dout_i, out_i> (fp32), also written for the dK/dV kernel
       float Di = 0.f, lse2 = INFINITY;
       if (valid) {
+        const int64_t r = bwd_row<MODE>(p, b, a, p.H, h, qrow);
         const uint4 *po = reinterpret_cast<const uint4 *>(p.out + r * D);
         const uint4 *pg = reinterpret_cast<const uint4 *>(p.dout + r * D);
         float2 acc = make_float2(0.f, 0.f);
@@ -356,11 +431,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
         Di = acc.x + acc.y;
-        p.delta[r] = Di;
-        lse2 = p.lse[r] * 1.4426950408889634f;
+        const int64_t rv = bwd_vec<MODE>(p, b, a, h, qrow);
+        p.delta[rv] = Di;
+        lse2 = p.lse[rv] * 1.4426950408889634f;
       }
       for (int j = 0; j < n; ++j) {
-        const int kt = k_lo + j;
+        const int kt = tl.kt(j);
         const int x = j & 1;
         if (!mbar_wait_warp(BAR_SF + 8 * x, s_cnt[x] & 1, abort_flag)) {
           stop = true;
@@ -368,12 +444,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         ++s_cnt[x];
         tc_fence_after();
-        // allowed key columns of this row: positions in [qrow - W + 1, qrow] and < N
+        // allowed key columns of this row: positions in [qrow - W + 1, qrow] and
+        // < len, and with sinks the positions below n_sink (up to the row)
         const int c0 = kt * kBwdT;
         const bool full = c0 + kBwdT - 1 <= t * kBwdT && c0 >= t * kBwdT + kBwdT - p.W &&
-                          t * kBwdT + kBwdT <= p.N;
+                          t * kBwdT + kBwdT <= len;
         uint32_t mw[4];
-        col_mask(qrow - p.W + 1 - c0, min(qrow, p.N - 1) - c0, mw);
+        col_mask(qrow - p.W + 1 - c0, min(qrow, len - 1) - c0, mw);
+        if (SINK && c0 == 0) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            mw[w] |= range_bits(-32 * w, min(p.n_sink - 1, min(qrow, len - 1)) - 32 * w);
+        }
         const uint32_t tS = tmem + T_S + x * 128 + lane_off;
         const uint32_t tP = tmem + T_DP + lane_off;
         // phase 1 (needs only S): P in fp32
@@ -439,8 +521,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       {
         // rows of this lane's 8-lane group: whole 128-byte segments per store
         const int g_row = t * kBwdT + quad * 32 + (lane & ~7);
-        store_tile_rows<D>(p.dq + ((static_cast<int64_t>(b) * p.H + h) * p.N + g_row) * D, D,
-                           p.N - g_row, tmem + T_DQ + lane_off, p.scale, lane);
+        store_tile_rows<D>(p.dq + bwd_row<MODE>(p, b, a, p.H, h, g_row) * D,
+                           MODE == 2 ? static_cast<int64_t>(p.H) * D : D, len - g_row,
+                           tmem + T_DQ + lane_off, p.scale, lane);
       }
       tc_fence_before();
       mbar_arrive(BAR_DQE);
@@ -458,7 +541,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // -------------------------------------------------------------------------------- dK dV
 // Unit u: (b, kv head, key tile kt); steps over (query head g of the group, live
 // query tile t in [kt, t_hi]).
-template <int D>
+template <int D, int MODE, bool SINK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -524,14 +607,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // tensor memory: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D)
   const uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 
-  // unit -> (b, kv head, kt); query tiles [kt, t_hi] of each of the G heads
-  auto unit = [&](int u, int &b, int &kvh, int &kt, int &t_hi) {
+  // unit -> (b, kv head, kt) and its sequence; query tiles [kt, t_hi] of each
+  // of the G heads (all of the sequence's for the key tile of the sinks).
+  // 0: run it, 1: bad sequence offsets (skip, flag), 2: the key tile lies past
+  // the sequence's end (skip).  Key tile 0 of every (b, kv head) first, then
+  // key tile 1, and so on: the heaviest units first (with sinks, key tile 0
+  // is read by every query tile of its sequence).
+  auto unit = [&](int u, int &b, int &kvh, int &kt, int &t_hi, int64_t &a, int &len) -> int {
     const int per_t = p.B * p.Hkv;
     kt = u / per_t;
     const int bk = u % per_t;
     b = bk / p.Hkv;
     kvh = bk % p.Hkv;
-    t_hi = min(p.nt - 1, (kt * kBwdT + kBwdT - 1 + p.W - 1) / kBwdT);
+    if (bwd_seq<MODE>(p, b, a, len)) return 1;
+    if (kt * kBwdT >= len) return 2;
+    const int nt_s = (len + kBwdT - 1) / kBwdT;
+    t_hi = (SINK && p.n_sink > 0 && kt == 0)
+               ? nt_s - 1
+               : min(nt_s - 1, (kt * kBwdT + kBwdT - 1 + p.W - 1) / kBwdT);
+    return 0;
   };
   auto unit_of = [&](int i) -> int {
     const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
@@ -543,20 +637,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       int u_iter = 0, q_iter = 0;
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        int b, kvh, kt, t_hi;
-        unit(u, b, kvh, kt, t_hi);
+        int b, kvh, kt, t_hi, len;
+        int64_t a;
+        const int ust = unit(u, b, kvh, kt, t_hi, a, len);
+        if (ust) {
+          if (ust == 1) atomicOr(&g_swa_status, SWA_DEV_BADARG);
+          continue;
+        }
         if (u_iter > 0 && !mbar_wait(BAR_KVE, (u_iter - 1) & 1, abort_flag)) break;
         mbar_expect_tx(BAR_KVF, 2 * L::TILE);
-        const int zk = b * p.Hkv + kvh;
+        // MODE 2 maps are {D, heads, tokens}: (head, token) replace (row, plane)
+        const int ky = MODE == 2 ? kvh : kt * kBwdT;
+        const int kz = MODE == 2 ? static_cast<int>(a) + kt * kBwdT : b * p.Hkv + kvh;
 #pragma unroll
         for (int pn = 0; pn < L::PANELS; ++pn) {
-          tma_load_3d(sK + pn * (kBwdT * 128), &tm_k, BAR_KVF, pn * 64, kt * kBwdT, zk);
-          tma_load_3d(sV + pn * (kBwdT * 128), &tm_v, BAR_KVF, pn * 64, kt * kBwdT, zk);
+          tma_load_3d(sK + pn * (kBwdT * 128), &tm_k, BAR_KVF, pn * 64, ky, kz);
+          tma_load_3d(sV + pn * (kBwdT * 128), &tm_v, BAR_KVF, pn * 64, ky, kz);
         }
         ++u_iter;
         for (int g = 0; g < p.G; ++g) {
-          const int zq = b * p.H + kvh * p.G + g;
+          const int hq = kvh * p.G + g;
           for (int t = kt; t <= t_hi; ++t) {
+            const int qy = MODE == 2 ? hq : t * kBwdT;
+            const int qz = MODE == 2 ? static_cast<int>(a) + t * kBwdT : b * p.H + hq;
             const int st = q_iter % NS;
             if (q_iter >= NS && !mbar_wait(BAR_QE + 8 * st, ((q_iter / NS) - 1) & 1, abort_flag))
               break;
@@ -564,9 +667,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int pn = 0; pn < L::PANELS; ++pn) {
               tma_load_3d(sQ + st * L::TILE + pn * (kBwdT * 128), &tm_q, BAR_QF + 8 * st, pn * 64,
-                          t * kBwdT, zq);
+                          qy, qz);
               tma_load_3d(sDO + st * L::TILE + pn * (kBwdT * 128), &tm_do, BAR_QF + 8 * st,
-                          pn * 64, t * kBwdT, zq);
+                          pn * 64, qy, qz);
             }
             ++q_iter;
           }
@@ -603,8 +706,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  (acc || kk > 0) ? 1u : 0u);
       };
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-        int b, kvh, kt, t_hi;
-        unit(u, b, kvh, kt, t_hi);
+        int b, kvh, kt, t_hi, len;
+        int64_t a;
+        if (unit(u, b, kvh, kt, t_hi, a, len)) continue;
         const int n = p.G * (t_hi - kt + 1);
         if (!mbar_wait(BAR_KVF, u_iter & 1, abort_flag)) break;
         tc_fence_after();
@@ -665,17 +769,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t s_cnt = 0, u_iter = 0, step = 0;
     for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
-      int b, kvh, kt, t_hi;
-      unit(u, b, kvh, kt, t_hi);
+      int b, kvh, kt, t_hi, len;
+      int64_t a;
+      if (unit(u, b, kvh, kt, t_hi, a, len)) continue;
       const int krow = kt * kBwdT + row;
       const int nqt = t_hi - kt + 1, n = p.G * nqt;
+      // query columns this key row reaches: [krow, krow + W - 1] (a sink row:
+      // every later one) within the sequence; none for rows past its end
+      const int qhi = (SINK && krow < p.n_sink) ? len - 1 : min(krow + p.W - 1, len - 1);
       // lse2 and D of query column et of step s: (query head g, query tile t)
       auto col_vals = [&](int s, float &l2, float &dd) {
         const int g = s / nqt, t = kt + s % nqt;
-        const int64_t rb = (static_cast<int64_t>(b) * p.H + kvh * p.G + g) * p.N;
         const int qc = t * kBwdT + et;
-        l2 = qc < p.N ? p.lse[rb + qc] * 1.4426950408889634f : INFINITY;
-        dd = qc < p.N ? p.delta[rb + qc] : 0.f;
+        const int64_t rv = bwd_vec<MODE>(p, b, a, kvh * p.G + g, qc);
+        l2 = qc < len ? p.lse[rv] * 1.4426950408889634f : INFINITY;
+        dd = qc < len ? p.delta[rv] : 0.f;
       };
       // stage a step's 128 (lse2, D) column values (two copies alternate).  Step
       // s + 1 is staged at the end of step s, after this thread's last read of
@@ -701,28 +809,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         tc_fence_after();
-        // allowed query columns of key row krow: i in [krow, krow + W - 1], i < N
+        // allowed query columns of key row krow (see qhi above)
         const int c0 = t * kBwdT;
         const bool full = kt * kBwdT + kBwdT - 1 <= c0 && c0 + kBwdT - 1 - kt * kBwdT <= p.W - 1 &&
-                          c0 + kBwdT <= p.N;
+                          c0 + kBwdT <= len;
         uint32_t mw[4];
-        col_mask(krow - c0, min(krow + p.W - 1, p.N - 1) - c0, mw);
+        col_mask(krow - c0, qhi - c0, mw);
         const uint32_t tS = tmem + T_S + lane_off;
         const uint32_t tP = tmem + T_DP + lane_off;
-        // phase 1: P^T (fp32 kept for dS), stored as bf16 over the low half of S^T
-        float pf[kBwdT];
+        // phase 1: P^T, stored as bf16 over the low half of S^T and kept for dS:
+        // in fp32 on the [B, heads, N, d] layout; on the packed layout, whose
+        // wider addressing leaves no room for a 128-register row, as the bf16
+        // pairs just stored (the same rounded P that dV uses)
+        constexpr bool kPackedP = MODE == 2;
+        float pf[kPackedP ? 1 : kBwdT];
+        uint32_t pw[kPackedP ? kBwdT / 2 : 1];
         auto pchunk = [&](int ch, const uint32_t (&sr)[32]) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
+            float pr[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int c = 2 * i + e;
-              float pr = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -v2[ch * 32 + c]));
-              if (!full && !((mw[ch] >> c) & 1u)) pr = 0.f;
-              pf[ch * 32 + c] = pr;
+              pr[e] = ex2(fmaf(__uint_as_float(sr[c]), p.scale_log2, -v2[ch * 32 + c]));
+              if (!full && !((mw[ch] >> c) & 1u)) pr[e] = 0.f;
+              if (!kPackedP) pf[ch * 32 + c] = pr[e];
             }
-            pk[i] = pack_bf16(pf[ch * 32 + 2 * i], pf[ch * 32 + 2 * i + 1]);
+            pk[i] = pack_bf16(pr[0], pr[1]);
+            if (kPackedP) pw[ch * 16 + i] = pk[i];
           }
           tmem_st16_b(tS + ch * 16, pk);
         };
@@ -757,7 +872,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int c = 2 * i + e;
-              dd[e] = pf[ch * 32 + c] * (__uint_as_float(dr[c]) - v2[kBwdT + ch * 32 + c]);
+              float pe;
+              if (kPackedP) {
+                const uint32_t w = pw[ch * 16 + i];
+                pe = __uint_as_float(e ? (w & 0xFFFF0000u) : (w << 16));
+              } else {
+                pe = pf[ch * 32 + c];
+              }
+              dd[e] = pe * (__uint_as_float(dr[c]) - v2[kBwdT + ch * 32 + c]);
             }
             dk[i] = pack_bf16(dd[0], dd[1]);
           }
@@ -787,9 +909,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       // rows of this lane's 8-lane group: whole 128-byte segments per store
       const int g_row = kt * kBwdT + quad * 32 + (lane & ~7);
-      const int64_t g_off = ((static_cast<int64_t>(b) * p.Hkv + kvh) * p.N + g_row) * D;
-      store_tile_rows<D>(p.dv + g_off, D, p.N - g_row, tmem + T_DV + lane_off, 1.f, lane);
-      store_tile_rows<D>(p.dk + g_off, D, p.N - g_row, tmem + T_DK + lane_off, p.scale, lane);
+      const int64_t g_off = bwd_row<MODE>(p, b, a, p.Hkv, kvh, g_row) * D;
+      const int64_t g_stride = MODE == 2 ? static_cast<int64_t>(p.Hkv) * D : D;
+      store_tile_rows<D>(p.dv + g_off, g_stride, len - g_row, tmem + T_DV + lane_off, 1.f, lane);
+      store_tile_rows<D>(p.dk + g_off, g_stride, len - g_row, tmem + T_DK + lane_off, p.scale,
+                         lane);
       tc_fence_before();
       mbar_arrive(BAR_AE);
     }

@@ -511,24 +511,30 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
       constexpr uint32_t idO = idesc_bf16_f32(kQT, D, true);
       int kv_iter = 0, q_iter = 0;
       uint32_t p_cnt[2] = {0u, 0u};
+      // Shared-memory descriptors as (low word + offset >> 4, constant high
+      // word): one 32-bit add per MMA.  The empty asm keeps the compiler from
+      // precomputing every MMA's words for the whole loop, which would spill.
+      constexpr uint32_t kDescHi = sdesc_sw128_hi(1024);
+      const uint32_t q_lo[2] = {sdesc_sw128_lo(sQ[0], 16), sdesc_sw128_lo(sQ[1], 16)};
+      const uint32_t k_lo = sdesc_sw128_lo(sK, 16), v_lo = sdesc_sw128_lo(sV, kKT * 128);
       auto issue_s = [&](int x, int st) {
-        const uint32_t dS = tmem + x * 128;
+        uint32_t qb = q_lo[x], kb = k_lo + st * (L::KV_BYTES >> 4), dS = tmem + x * 128;
+        asm volatile("" : "+r"(qb), "+r"(kb), "+r"(dS));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t offq = (kk >> 2) * (kQT * 128) + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * (kKT * 128) + (kk & 3) * 32;
-          mma_ss(dS, sdesc_sw128(sQ[x] + offq, 16, 1024),
-                 sdesc_sw128(sK + st * L::KV_BYTES + offk, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          mma_ss_w(dS, qb + (offq >> 4), kb + (offk >> 4), kDescHi, idS, kk > 0 ? 1u : 0u);
         }
         tc_commit(BAR_S + 8 * x);
       };
       auto issue_pv = [&](int x, int st, bool acc) {
-        const uint32_t dO = tmem + 256 + x * D;
-        const uint32_t aP = tmem + x * 128;
+        uint32_t dO = tmem + 256 + x * D, aP = tmem + x * 128, vb = v_lo + st * (L::KV_BYTES >> 4);
+        asm volatile("" : "+r"(vb), "+r"(dO), "+r"(aP));
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          mma_ts(dO, aP + kk * 8, sdesc_sw128(sV + st * L::KV_BYTES + kk * 16 * 128, kKT * 128, 1024),
-                 idO, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_w(dO, aP + kk * 8, vb + ((kk * 16 * 128) >> 4), kDescHi, idO,
+                   (acc || kk > 0) ? 1u : 0u);
       };
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         Unit U = decode_unit(u, p);

@@ -511,12 +511,12 @@ size_t swa_attn_bwd_workspace_bytes(int B, int H, int64_t N) {
 }  // extern "C"
 
 namespace {
-template <int D>
+template <int D, int MODE, bool SINK>
 int launch_bwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                const CUtensorMap &tdo, swa::BwdParams p, cudaStream_t st) {
   using L = swa::BwdLayout<D>;
-  auto kq = swa::bwd_dq_kernel<D>;
-  auto kkv = swa::bwd_dkdv_kernel<D>;
+  auto kq = swa::bwd_dq_kernel<D, MODE, SINK>;
+  auto kkv = swa::bwd_dkdv_kernel<D, MODE, SINK>;
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
           cudaSuccess ||
       cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
@@ -538,14 +538,11 @@ int launch_bwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
                                                                                   p);
   return check_launch();
 }
-}  // namespace
 
-extern "C" {
-
-int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
-                 const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int64_t N,
-                 int d, int64_t W, float scale, void *workspace, size_t workspace_bytes,
-                 void *stream) {
+int attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+             const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int64_t N,
+             int d, int64_t W, int n_sink, float scale, void *workspace, size_t workspace_bytes,
+             void *stream) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return SWA_ERR_INVALID_ARG;
@@ -553,6 +550,7 @@ int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return SWA_ERR_INVALID_ARG;
   if (N < 1 || N >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_sink > kBK) return SWA_ERR_INVALID_ARG;
   const size_t need = swa_attn_bwd_workspace_bytes(B, H, N);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SWA_ERR_WORKSPACE;
   CUtensorMap tq, tk, tv, tdo;
@@ -577,8 +575,87 @@ int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.nt = static_cast<int>((N + swa::kBwdT - 1) / swa::kBwdT);
+  p.n_sink = n_sink;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_bwd<128>(tq, tk, tv, tdo, p, st) : launch_bwd<64>(tq, tk, tv, tdo, p, st);
+  if (n_sink > 0)
+    return d == 128 ? launch_bwd<128, 0, true>(tq, tk, tv, tdo, p, st)
+                    : launch_bwd<64, 0, true>(tq, tk, tv, tdo, p, st);
+  return d == 128 ? launch_bwd<128, 0, false>(tq, tk, tv, tdo, p, st)
+                  : launch_bwd<64, 0, false>(tq, tk, tv, tdo, p, st);
+}
+}  // namespace
+
+extern "C" {
+
+int swa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int64_t N,
+                 int d, int64_t W, float scale, void *workspace, size_t workspace_bytes,
+                 void *stream) {
+  return attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, Hkv, N, d, W, 0, scale, workspace,
+                  workspace_bytes, stream);
+}
+
+int swa_attn_bwd_sink(const void *q, const void *k, const void *v, const void *out,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                      int H, int Hkv, int64_t N, int d, int64_t W, int n_sink, float scale,
+                      void *workspace, size_t workspace_bytes, void *stream) {
+  return attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, Hkv, N, d, W, n_sink, scale,
+                  workspace, workspace_bytes, stream);
+}
+
+size_t swa_attn_varlen_bwd_workspace_bytes(int H, int64_t total) {
+  if (H < 1 || total < 1) return 0;
+  return align256(static_cast<size_t>(H) * static_cast<size_t>(total) * sizeof(float));
+}
+
+int swa_attn_varlen_bwd(const void *q, const void *k, const void *v, const int64_t *cu_seqlens,
+                        const void *out, const void *dout, const float *lse, void *dq, void *dk,
+                        void *dv, int n_seq, int64_t total, int64_t max_seqlen, int H, int Hkv,
+                        int d, int64_t W, int n_sink, float scale, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+  int e = common_checks(n_seq, H, Hkv, d, W, scale);
+  if (e) return e;
+  if (!q || !k || !v || !cu_seqlens || !out || !dout || !lse || !dq || !dk || !dv)
+    return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SWA_ERR_INVALID_ARG;
+  if (total < 1 || total >= (int64_t(1) << 31) - 2 * kBQ) return SWA_ERR_INVALID_ARG;
+  if (max_seqlen < 1 || max_seqlen >= (int64_t(1) << 29)) return SWA_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_sink > kBK) return SWA_ERR_INVALID_ARG;
+  const size_t need = swa_attn_varlen_bwd_workspace_bytes(H, total);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SWA_ERR_WORKSPACE;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((e = make_map_tokens(&tq, q, d, H, total, swa::kBwdT))) return e;
+  if ((e = make_map_tokens(&tk, k, d, Hkv, total, swa::kBwdT))) return e;
+  if ((e = make_map_tokens(&tv, v, d, Hkv, total, swa::kBwdT))) return e;
+  if ((e = make_map_tokens(&tdo, dout, d, H, total, swa::kBwdT))) return e;
+  swa::BwdParams p;
+  p.out = static_cast<const __nv_bfloat16 *>(out);
+  p.dout = static_cast<const __nv_bfloat16 *>(dout);
+  p.lse = lse;
+  p.delta = static_cast<float *>(workspace);
+  p.dq = static_cast<__nv_bfloat16 *>(dq);
+  p.dk = static_cast<__nv_bfloat16 *>(dk);
+  p.dv = static_cast<__nv_bfloat16 *>(dv);
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
+  p.n_sink = n_sink;
+  p.B = n_seq;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.N = static_cast<int>(max_seqlen);
+  p.W = static_cast<int>(W < max_seqlen + swa::kBwdT ? W : max_seqlen + swa::kBwdT);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nt = static_cast<int>((max_seqlen + swa::kBwdT - 1) / swa::kBwdT);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_sink > 0)
+    return d == 128 ? launch_bwd<128, 2, true>(tq, tk, tv, tdo, p, st)
+                    : launch_bwd<64, 2, true>(tq, tk, tv, tdo, p, st);
+  return d == 128 ? launch_bwd<128, 2, false>(tq, tk, tv, tdo, p, st)
+                  : launch_bwd<64, 2, false>(tq, tk, tv, tdo, p, st);
 }
 
 int swa_ring_slot_positions(int B, const int64_t *n_written, int64_t W, int64_t *slot_pos,

@@ -70,6 +70,9 @@ WORKLOADS = {
     "chunk_ring_sink": Workload("chunk_ring_sink", "chunk", B=4, H=32, Hkv=8, d=128, W=4096,
                                 Tq=512, q_start=12288, n_sink=4, seed=10,
                                 note="chunked prefill on a ring cache with 4 attention sinks"),
+    "varlen_backward": Workload("varlen_backward", "varlen_backward", B=1, H=32, Hkv=8, d=128,
+                                W=4096, n_seq=16, len_lo=256, len_hi=16384, n_sink=4, seed=11,
+                                note="gradients of 16 packed sequences with 4 sinks"),
     "mistral_backward": Workload("mistral_backward", "backward", B=1, H=32, Hkv=8, d=128, W=4096,
                                  N=8192, seed=9, note="gradients of the Mistral-shaped prefill"),
 }
@@ -77,7 +80,7 @@ WORKLOADS = {
 
 def seq_lens(w: Workload) -> np.ndarray:
     """Packed sequence lengths (varlen) or valid chunk rows per sequence (ragged chunk)."""
-    count = w.n_seq if w.kind == "varlen" else w.B
+    count = w.n_seq if w.kind in ("varlen", "varlen_backward") else w.B
     return uniform_int(w.seed, STREAM["seq_len"], count, w.len_lo, w.len_hi)
 
 

@@ -81,6 +81,12 @@ def test_varlen_counts():
     lens = [int(x) for x in seq_lens(v)]
     assert len(lens) == 16 and all(256 <= x <= 16384 for x in lens)
     assert bench.useful_flops(v) == 4 * 128 * 32 * sum(bench.sequence_pairs(n, 4096) for n in lens)
+    # the packed backward: five products per visible pair (window and sinks), per sequence
+    vb = WORKLOADS["varlen_backward"]
+    lens_b = [int(x) for x in seq_lens(vb)]
+    assert len(lens_b) == 16 and all(256 <= x <= 16384 for x in lens_b)
+    assert bench.useful_flops(vb) == 10 * 128 * 32 * sum(oracle.count_pairs_sink(n, 4096, 4)
+                                                         for n in lens_b)
 
 
 def test_decode_bytes():

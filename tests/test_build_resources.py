@@ -81,6 +81,6 @@ def test_headline_forward_kernels_do_not_spill(report):
 
 def test_backward_kernels_fit_their_block(report):
     bwd = {n: r for n, r in report.items() if "bwd_dq_kernel" in n or "bwd_dkdv_kernel" in n}
-    assert len(bwd) == 4
+    assert len(bwd) == 16          # 2 kernels x D in {64, 128} x layout {0, 2} x SINK
     for name, r in bwd.items():
         assert r.get("regs", 0) <= 255, (name, r)
