@@ -17,7 +17,10 @@
 //                 S_X = Q_X K^T        (A, B from shared memory)
 //                 O_X += P_X V         (P from tensor memory, V from shared memory)
 //               in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
-//               softmax of one tile overlaps the MMAs of the other.
+//               softmax of one tile overlaps the MMAs of the other.  On the
+//               linear and packed layouts the softmax hands P over in two
+//               halves of 64 keys, and the PV of the first half runs while the
+//               exponentials of the second are computed.
 //   warps 2-3   idle (they complete warpgroup 0).
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one row per
 //               thread, one tensor-memory lane quadrant per warp.  Mask only
@@ -101,8 +104,8 @@ struct Fwd2Layout {
   static constexpr uint32_t OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + NV * KV_BYTES;
   // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
-  // o_full[2], mma_drain
-  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 7;
+  // o_full[2], mma_drain, p2_full[2]
+  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 9;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t BYTES = OFF_MISC + 16;
   static constexpr uint32_t ALLOC = BYTES + 1024;
@@ -351,6 +354,12 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
   const uint32_t BAR_P = BAR_S + 16;                // + 8 * tile
   const uint32_t BAR_O = BAR_P + 16;                // + 8 * tile
   const uint32_t BAR_DRAIN = BAR_O + 16;            // the MMA thread's teardown
+  const uint32_t BAR_P2 = BAR_DRAIN + 8;            // + 8 * tile: second half of P stored
+  // P is handed to the PV MMA in two halves of 64 keys (the first half's PV
+  // runs while the softmax computes the second), except on the ring layout,
+  // whose MMA thread already does more per tile (there the split measured
+  // 2% slower; on the linear and packed layouts 3-6% faster).
+  constexpr bool kSplitP = MODE != 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -369,6 +378,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(BAR_S + 8 * x, 1);
       mbar_init(BAR_P + 8 * x, 4 * 32);
+      mbar_init(BAR_P2 + 8 * x, 4 * 32);
       mbar_init(BAR_O + 8 * x, 1);
     }
     mbar_init(BAR_DRAIN, 1);
@@ -528,13 +538,28 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         }
         tc_commit(BAR_S + 8 * x);
       };
-      auto issue_pv = [&](int x, int st, bool acc) {
+      // PV over keys k_begin .. k_begin + n_keys - 1 of the tile
+      auto issue_pv = [&](int x, int st, bool acc, int k_begin, int n_keys) {
         uint32_t dO = tmem + 256 + x * D, aP = tmem + x * 128, vb = v_lo + st * (L::KV_BYTES >> 4);
         asm volatile("" : "+r"(vb), "+r"(dO), "+r"(aP));
 #pragma unroll
-        for (int kk = 0; kk < kKT / 16; ++kk)
+        for (int k16 = 0; k16 < n_keys / 16; ++k16) {
+          const int kk = k_begin / 16 + k16;
           mma_ts_w(dO, aP + kk * 8, vb + ((kk * 16 * 128) >> 4), kDescHi, idO,
                    (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      // P_X of one tile: in two halves (kSplitP), or whole; false if a wait gave up
+      auto pv_tile = [&](int x, int st, bool acc) -> bool {
+        if (kSplitP) {
+          issue_pv(x, st, acc, 0, kKT / 2);
+          if (!mbar_wait(BAR_P2 + 8 * x, p_cnt[x] & 1, abort_flag)) return false;
+          tc_fence_after();
+          issue_pv(x, st, true, kKT / 2, kKT / 2);
+        } else {
+          issue_pv(x, st, acc, 0, kKT);
+        }
+        return true;
       };
       for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
         Unit U = decode_unit(u, p);
@@ -588,9 +613,12 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
               stop = true;
               break;
             }
-            ++p_cnt[0];
             tc_fence_after();
-            issue_pv(0, sv, !first[0]);
+            if (!pv_tile(0, sv, !first[0])) {
+              stop = true;
+              break;
+            }
+            ++p_cnt[0];
             first[0] = false;
             // linear keys: a query tile's live tiles are contiguous, so it is done
             // (tile A's stay so with the sink tile in front; B's need not)
@@ -612,9 +640,12 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
               stop = true;
               break;
             }
-            ++p_cnt[1];
             tc_fence_after();
-            issue_pv(1, sv, !first[1]);
+            if (!pv_tile(1, sv, !first[1])) {
+              stop = true;
+              break;
+            }
+            ++p_cnt[1];
             first[1] = false;
             if (b_contig && !(has_next && nb)) {
               tc_commit(BAR_O + 8);
@@ -731,43 +762,72 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         float2 *s2 = reinterpret_cast<float2 *>(s);
 #pragma unroll
         for (int c = 0; c < kKT / 2; ++c) s2[c] = __ffma2_rn(s2[c], sc2, nm2);
-        // exponentials on the MUFU (a masked column gives 2^-inf = 0)
-#pragma unroll
-        for (int c = 0; c < kKT; ++c) s[c] = ex2(s[c]);
-        float2 sm2[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kKT / 2; c += 4)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sm2[i] = __fadd2_rn(sm2[i], s2[c + i]);
-        const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
-        const float rs = sa.x + sa.y;
-        l_run = l_run * alpha + rs;
-        m_run = m_new;
-        // P (bf16 pairs, key 2c in the low half of column c) over the first 64 columns of S_X
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
+        // P of keys 64h .. 64h + 63 as bf16 pairs (key 2c in the low half of
+        // column c) into columns 32h .. 32h + 31 of S_X; no wait
+        auto store_p = [&](int h) {
           uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[h2 * 64 + 2 * i], s[h2 * 64 + 2 * i + 1]);
-          tmem_st32(tS + h2 * 32, pk);
-        }
-        // O_X is stable: PV_X of the previous tile was issued before this S_X
-        if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]);
+          tmem_st32(tS + h * 32, pk);
+        };
+        auto rescale_o = [&](float a) {
 #pragma unroll 1
           for (int cb2 = 0; cb2 < D / 32; ++cb2) {
             uint32_t o32[32];
             tmem_ld32(tO + cb2 * 32, o32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * a);
             tmem_st32(tO + cb2 * 32, o32);
           }
+        };
+        if (kSplitP) {
+          // O_X is stable (PV_X of the previous tile was issued before this
+          // S_X): rescale it before the first half of P hands PV_X the tile
+          if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o(alpha);
+          // exponentials on the MUFU (a masked column gives 2^-inf = 0) in two
+          // halves of 64 keys; P of the first half (bf16 pairs, key 2c in the
+          // low half of column c) goes to PV_X while the second is computed
+          float2 sm2[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+            for (int c = h2 * 64; c < h2 * 64 + 64; ++c) s[c] = ex2(s[c]);
+#pragma unroll
+            for (int c = h2 * 32; c < h2 * 32 + 32; c += 4)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) sm2[i] = __fadd2_rn(sm2[i], s2[c + i]);
+            store_p(h2);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(h2 == 0 ? BAR_P + 8 * x : BAR_P2 + 8 * x);
+          }
+          const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
+          l_run = l_run * alpha + (sa.x + sa.y);
+          m_run = m_new;
+        } else {
+          // exponentials on the MUFU (a masked column gives 2^-inf = 0)
+#pragma unroll
+          for (int c = 0; c < kKT; ++c) s[c] = ex2(s[c]);
+          float2 sm2[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sm2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < kKT / 2; c += 4)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sm2[i] = __fadd2_rn(sm2[i], s2[c + i]);
+          const float2 sa = __fadd2_rn(__fadd2_rn(sm2[0], sm2[1]), __fadd2_rn(sm2[2], sm2[3]));
+          l_run = l_run * alpha + (sa.x + sa.y);
+          m_run = m_new;
+          store_p(0);
+          store_p(1);
+          // O_X is stable: PV_X of the previous tile was issued before this S_X
+          if (nt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o(alpha);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(BAR_P + 8 * x);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(BAR_P + 8 * x);
         ++nt;
       }
       if (stop) break;
