@@ -373,9 +373,13 @@ def make_call(w, x, swa):
     if w.kind == "chunk":
         out = torch.empty_like(x["q"])
         if "chunk_len" in x:
-            return (lambda: swa.swa_attn_chunk_ring_ragged(
-                x["q"], x["k_new"], x["v_new"], x["k_ring"], x["v_ring"], x["q_start"],
-                x["chunk_len"], w.scale, out=out), out, 1)
+            # ragged chunks leave the last round of units part empty: the split call
+            # (schedule, attention, merge) cuts those units by key range across the SMs
+            ws = torch.empty(swa.swa_chunk_split_workspace_bytes(w.B, w.H, w.Hkv, w.Tq, w.d, w.W),
+                             dtype=torch.uint8, device=x["q"].device)
+            return (lambda: swa.swa_attn_chunk_ring_split(
+                x["q"], x["k_new"], x["v_new"], x["k_ring"], x["v_ring"], x["q_start"], w.scale,
+                chunk_len=x["chunk_len"], out=out, workspace=ws), out, 3)
         return (lambda: swa.swa_attn_chunk_ring(x["q"], x["k_new"], x["v_new"], x["k_ring"],
                                                 x["v_ring"], x["q_start"], w.scale, out=out,
                                                 k_sink=x.get("k_sink"), v_sink=x.get("v_sink")),

@@ -313,6 +313,45 @@ SWA_API int swa_attn_chunk_ring_ragged(const void *q, const void *k_new, const v
                                        int update_ring, void *stream);
 
 /*
+ * swa_chunk_split_workspace_bytes -- bytes of scratch swa_attn_chunk_ring_split
+ * needs for these sizes on the current device (its SM count sets how many
+ * parts a call can have), 256-byte aligned; 0 for invalid sizes.
+ */
+SWA_API size_t swa_chunk_split_workspace_bytes(int B, int H, int Hkv, int64_t Tq, int d,
+                                               int64_t W);
+
+/*
+ * swa_attn_chunk_ring_split -- the chunked prefill over a ring of
+ * swa_attn_chunk_ring, swa_attn_chunk_ring_ragged and swa_attn_chunk_ring_sink
+ * in one call, with a caller workspace that lets it balance its work.
+ * Passage: Chapter 10 section 10.2 (each query of a chunk attends to its own
+ * window over the ring and chunk keys; splitting that key set changes only
+ * how the softmax is summed).  Every two-query-tile unit of a chunk reads
+ * about the same number of key tiles, so when the live units (those whose
+ * rows hold valid chunk rows) leave the last round of units on the SMs part
+ * empty -- a batch of short or few chunks -- each unit of that round is cut
+ * into parts over its key tiles, one per SM; the parts write unnormalised
+ * rows with their running max and sum to the workspace and a merge kernel
+ * combines them (as the decode path merges its splits).  Results equal the
+ * unsplit call's within rounding (a different summation order).
+ *   k_sink, v_sink, n_sink: as swa_attn_chunk_ring_sink, or NULL, NULL, 0.
+ *   chunk_len: as swa_attn_chunk_ring_ragged, or NULL (every chunk Tq rows).
+ *   workspace: device scratch of at least swa_chunk_split_workspace_bytes(B,
+ *      H, Hkv, Tq, d, W) bytes, 256-byte aligned, caller-owned; contents on
+ *      entry are ignored (SWA_ERR_WORKSPACE if missing, small or unaligned).
+ * Other arguments, layouts, limits and the ring update as swa_attn_chunk_ring.
+ * Three kernels on `stream` (schedule, attention, merge), then the ring
+ * update when update_ring != 0.
+ */
+SWA_API int swa_attn_chunk_ring_split(const void *q, const void *k_new, const void *v_new,
+                                      void *k_ring, void *v_ring, const void *k_sink,
+                                      const void *v_sink, int n_sink, const int64_t *q_start,
+                                      const int64_t *chunk_len, void *out, float *lse, int B,
+                                      int H, int Hkv, int64_t Tq, int d, int64_t W, float scale,
+                                      int update_ring, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
+/*
  * swa_ring_write -- append a chunk of keys/values to a ring cache.
  * Passage: blog section 3.2 (slot = position mod W once the ring is full);
  * M003 note section 06 (update the position-to-slot map before reuse).

@@ -36,6 +36,8 @@ __all__ = [
     "swa_attn_chunk_ring",
     "swa_attn_chunk_ring_ragged",
     "swa_attn_chunk_ring_sink",
+    "swa_attn_chunk_ring_split",
+    "swa_chunk_split_workspace_bytes",
     "swa_ring_write",
     "swa_decode_workspace_bytes",
     "swa_attn_decode_ring",
@@ -301,6 +303,53 @@ def swa_attn_chunk_ring_ragged(q, k_new, v_new, k_ring, v_ring, q_start, chunk_l
                                            _ptr(v_ring), _ptr(q_start), _ptr(chunk_len),
                                            _ptr(out), _ptr(lse), B, H, Hkv, Tq, d, W, scale,
                                            1 if update_ring else 0, _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def swa_chunk_split_workspace_bytes(B: int, H: int, Hkv: int, Tq: int, d: int, W: int) -> int:
+    return int(lib().swa_chunk_split_workspace_bytes(B, H, Hkv, Tq, d, W))
+
+
+def swa_attn_chunk_ring_split(q, k_new, v_new, k_ring, v_ring, q_start, scale: float | None = None,
+                              chunk_len=None, k_sink=None, v_sink=None, update_ring: bool = False,
+                              out=None, lse=None, return_lse: bool = False, workspace=None):
+    """Chunked prefill on a ring cache with a workspace that balances the work.
+
+    The same results as swa_attn_chunk_ring / _ragged (chunk_len [B]) / _sink
+    (k_sink, v_sink [B,Hkv,S,d]), within rounding: the last round of units is
+    split across the SMs by key range and merged.  Rows past chunk_len[b] keep
+    what `out` held (zeros when allocated here).
+    """
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_ring, "k_ring"),
+                 (v_ring, "v_ring")):
+        _need(t, n, dims=4)
+    _need(q_start, "q_start", torch.int64, 1)
+    if chunk_len is not None:
+        _need(chunk_len, "chunk_len", torch.int64, 1)
+    n_sink = 0
+    if k_sink is not None:
+        _need(k_sink, "k_sink", dims=4)
+        _need(v_sink, "v_sink", dims=4)
+        n_sink = k_sink.shape[2]
+    B, H, Tq, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.zeros_like(q)
+    if return_lse and lse is None:
+        lse = torch.zeros((B, H, Tq), dtype=torch.float32, device=q.device)
+    need = swa_chunk_split_workspace_bytes(B, H, Hkv, Tq, d, W)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check("swa_attn_chunk_ring_split",
+          lib().swa_attn_chunk_ring_split(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring),
+                                          _ptr(v_ring), _ptr(k_sink), _ptr(v_sink), n_sink,
+                                          _ptr(q_start), _ptr(chunk_len), _ptr(out), _ptr(lse), B,
+                                          H, Hkv, Tq, d, W, scale, 1 if update_ring else 0,
+                                          _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

@@ -44,6 +44,9 @@ SIGNATURES = {
                                       _i, _i64, _f, _i, _p]),
     "swa_attn_chunk_ring_ragged": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i64, _i,
                                         _i64, _f, _i, _p]),
+    "swa_chunk_split_workspace_bytes": (_sz, [_i, _i, _i, _i64, _i, _i64]),
+    "swa_attn_chunk_ring_split": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _p, _i, _i, _i,
+                                       _i64, _i, _i64, _f, _i, _p, _sz, _p]),
     "swa_ring_write": (_i, [_p, _p, _p, _p, _p, _i, _i, _i64, _i, _i64, _p]),
     "swa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i64]),
     "swa_attn_decode_ring": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i64, _f, _p, _sz, _p]),

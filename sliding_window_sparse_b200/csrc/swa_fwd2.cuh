@@ -87,6 +87,13 @@ struct Fwd2Params {
   int n_ring_tiles = 0;    // MODE 1: ceil(W / kKT)
   int pair_heads = 0;      // 1: A/B are heads 2p, 2p+1 of a group; 0: q tiles 2p, 2p+1
   int n_units = 0;
+  // MODE 1 with split key ranges (swa_split.cuh): the per-CTA unit list
+  // [round * gridDim.x + cta] = {unit, part, parts, slot} (unit < 0 ends it),
+  // and the partial rows of the parts: running max and sum [slot][2][kQT][2],
+  // unnormalised O [slot][2][kQT][D].
+  const int4 *items = nullptr;
+  float *ws_ml = nullptr;
+  float *ws_o = nullptr;
 };
 
 template <int D>
@@ -166,9 +173,13 @@ struct Walker2 {
   bool sink_pending;  // the sink tile (MODE 0 / 2: key tile 0; MODE 1: the sink rows, k = -1)
                       // still to be yielded ahead of kt
   int sink_vis[2];    // MODE 1: sinks before the window of the tile's last row
+  int idx, t_lo, t_hi;  // MODE 1: stream index of the next live tile; the part's range
 
   // len: valid query rows of this unit's sequence (MODE 1: also its chunk keys)
   __device__ __forceinline__ void init(const Unit &U, const Fwd2Params &p, int64_t qs, int len) {
+    idx = 0;
+    t_lo = 0;
+    t_hi = 0x7FFFFFFF;
     has_b = U.has_b;
     n_k = MODE == 0 ? p.n_k : len;
     W = static_cast<int>(p.W);
@@ -284,9 +295,32 @@ struct Walker2 {
     return next(k, src, y0, ca, cb);
   }
 
+  // MODE 1, part `part` of `parts`: keep only the part's contiguous piece of
+  // the live tiles (by count), for a unit whose key range is split.
+  __device__ __forceinline__ void set_part(int part, int parts) {
+    if (parts <= 1) return;
+    Walker2 w = *this;
+    int n = 0, k, src, y0, ca, cb;
+    while (w.next_all(k, src, y0, ca, cb)) ++n;
+    t_lo = part * n / parts;
+    t_hi = (part + 1) * n / parts;
+  }
+
   // Advance to the next live tile: its index, source, first row and classes.
-  // Tile 0 under sinks is partial unless the window alone covers it.
+  // MODE 1 skips the tiles outside the part's range (set_part).
   __device__ __forceinline__ bool next(int &k, int &src, int &y0, int &ca, int &cb) {
+    if (MODE != 1) return next_all(k, src, y0, ca, cb);
+    while (next_all(k, src, y0, ca, cb)) {
+      const int i = idx++;
+      if (i < t_lo) continue;
+      return i < t_hi;
+    }
+    return false;
+  }
+
+  // Every live tile in stream order.  Tile 0 under sinks is partial unless
+  // the window alone covers it.
+  __device__ __forceinline__ bool next_all(int &k, int &src, int &y0, int &ca, int &cb) {
     int lo[2], hi[2], base[2];
     if (SINK && MODE == 1 && sink_pending) {
       sink_pending = false;
@@ -414,6 +448,23 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
     return i * P + ((i & 1) ? P - 1 - c : c);
   };
+  // The i-th unit of this CTA and which part of it (of `parts`; slot: the
+  // part's partial rows): from the split schedule's list when there is one.
+  auto item_of = [&](int i, int &u, int &part, int &parts, int &slot) -> bool {
+    if (MODE == 1 && p.items) {
+      const int4 v = p.items[static_cast<int64_t>(i) * gridDim.x + blockIdx.x];
+      u = v.x;
+      part = v.y;
+      parts = v.z;
+      slot = v.w;
+      return u >= 0;
+    }
+    u = unit_of(i);
+    part = 0;
+    parts = 1;
+    slot = -1;
+    return u < p.n_units;
+  };
 
   // 0: run the unit; 1: invalid start position, chunk length or sequence
   // offsets (skip, flag); 2: the unit's query rows are all padding of a
@@ -451,7 +502,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     if (lane == 0) {
       int kv_iter = 0, q_iter = 0;
       bool k_ahead = false;  // K of iteration kv_iter issued, its V not (abort between them)
-      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+      int u, part, parts, slot;
+      for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
         Unit U = decode_unit(u, p);
         int64_t qs;
         int len;
@@ -477,6 +529,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         ++q_iter;
         Walker2<MODE, SINK> wk;
         wk.init(U, p, qs, len);
+        wk.set_part(part, parts);
         int k, src, y0, ca, cb;
         // MODE 2 maps are {D, heads, tokens}: (head, token) replace (row, plane)
         const int z = MODE == 2 ? static_cast<int>(qs) : U.b * p.Hkv + U.kvh;
@@ -561,7 +614,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         }
         return true;
       };
-      for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+      int u, part, parts, slot;
+      for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
         Unit U = decode_unit(u, p);
         int64_t qs;
         int len;
@@ -570,6 +624,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         tc_fence_after();
         Walker2<MODE, SINK> wk;
         wk.init(U, p, qs, len);
+        wk.set_part(part, parts);
         int k, src, y0, ca, cb, na = 0, nb = 0;
         bool have = wk.next_live(k, src, y0, ca, cb);
         bool first[2] = {true, true};
@@ -688,13 +743,15 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     const uint32_t tO = tmem + 256 + x * D + lane_off;
     uint32_t s_cnt = 0, u_iter = 0;
     bool stop = false;  // a wait gave up (the whole warp): no more TMEM work or stores
-    for (int it = 0, u = unit_of(0); u < p.n_units; u = unit_of(++it)) {
+    int u, part, parts, slot;
+    for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
       Unit U = decode_unit(u, p);
       int64_t qs;
       int len;
       if (unit_start(U, qs, len)) continue;
       Walker2<MODE, SINK> wk;
       wk.init(U, p, qs, len);
+      wk.set_part(part, parts);
       // MODE 0 absolute, MODE 1 relative to q_start, MODE 2 within the sequence
       const int qrow = U.t[x] * kQT + row;
       float m_run = -INFINITY, l_run = 0.f;
@@ -831,7 +888,30 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         ++nt;
       }
       if (stop) break;
-      if (nt > 0) {
+      if (MODE == 1 && parts > 1) {
+        // one part of a split unit: this row's unnormalised O with its running
+        // max and sum, for the merge kernel (a row the part gave no key to
+        // gets sum 0, which the merge skips)
+        const int64_t r = (static_cast<int64_t>(slot) * 2 + x) * kQT + row;
+        if (nt > 0) {
+          if (!mbar_wait_warp(BAR_O + 8 * x, u_iter & 1, abort_flag)) break;
+          ++u_iter;
+          tc_fence_after();
+          float4 *po = reinterpret_cast<float4 *>(p.ws_o + r * D);
+#pragma unroll 1
+          for (int c32 = 0; c32 < D / 32; ++c32) {
+            uint32_t o32[32];
+            tmem_ld32(tO + c32 * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              po[c32 * 8 + i] = make_float4(__uint_as_float(o32[4 * i]), __uint_as_float(o32[4 * i + 1]),
+                                            __uint_as_float(o32[4 * i + 2]),
+                                            __uint_as_float(o32[4 * i + 3]));
+          }
+        }
+        p.ws_ml[2 * r] = m_run;
+        p.ws_ml[2 * r + 1] = nt > 0 ? l_run : 0.f;
+      } else if (nt > 0) {
         // every PV of this unit is done
         if (!mbar_wait_warp(BAR_O + 8 * x, u_iter & 1, abort_flag)) break;
         ++u_iter;

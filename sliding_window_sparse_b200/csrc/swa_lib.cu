@@ -21,6 +21,7 @@
 #include "swa_fwd2.cuh"
 #include "swa_meta.cuh"
 #include "swa_selftest.cuh"
+#include "swa_split.cuh"
 #include "swa_tile.cuh"
 
 namespace {
@@ -100,12 +101,29 @@ int common_checks(int B, int H, int Hkv, int d, int64_t W, float scale) {
   return SWA_OK;
 }
 
-// tks / tvs: the sink rows of the chunk-ring path with sinks (any map otherwise)
+// Work units of the forward: two query tiles that read the same key tiles
+// (two heads of a GQA group, or query tiles 2p and 2p + 1 of one head).
+int64_t fwd_units(swa::Fwd2Params &p) {
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  return p.pair_heads ? static_cast<int64_t>(p.B) * p.Hkv * (p.G / 2) * p.nqt
+                      : static_cast<int64_t>(p.B) * p.H * ((p.nqt + 1) / 2);
+}
+
+int sm_count(int *sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *sms < 1)
+    return SWA_ERR_CUDA;
+  return SWA_OK;
+}
+
+// tks / tvs: the sink rows of the chunk-ring path with sinks (any map otherwise).
+// full_grid: one CTA per SM whatever the unit count (the split schedule's P).
 template <int D, int MODE, bool SINK = false>
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                const CUtensorMap &tkr, const CUtensorMap &tvr, swa::Fwd2Params p,
                cudaStream_t st, const CUtensorMap *tks = nullptr,
-               const CUtensorMap *tvs = nullptr) {
+               const CUtensorMap *tvs = nullptr, bool full_grid = false) {
   using L = swa::Fwd2Layout<D>;
   auto kern = swa::fwd2_kernel<D, MODE, SINK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
@@ -124,17 +142,12 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
     launch_regs.store(regs, std::memory_order_relaxed);
   }
   if (regs != swa::kFwd2LaunchRegs) return SWA_ERR_UNSUPPORTED;
-  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
-  const int64_t units = p.pair_heads
-                            ? static_cast<int64_t>(p.B) * p.Hkv * (p.G / 2) * p.nqt
-                            : static_cast<int64_t>(p.B) * p.H * ((p.nqt + 1) / 2);
+  const int64_t units = fwd_units(p);
   if (units > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
   p.n_units = static_cast<int>(units);
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
-    return SWA_ERR_CUDA;
-  const int grid = static_cast<int>(units < sms ? units : sms);
+  int sms = 0;
+  if (sm_count(&sms)) return SWA_ERR_CUDA;
+  const int grid = full_grid ? sms : static_cast<int>(units < sms ? units : sms);
   kern<<<grid, swa::kFwd2Threads, L::ALLOC, st>>>(tq, tk, tv, tkr, tvr, tks ? *tks : tk,
                                                    tvs ? *tvs : tv, p);
   return check_launch();
@@ -182,6 +195,32 @@ int dispatch_decode_g(int G, const swa::DecodeParams &p, cudaStream_t st) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The chunk forward with its key ranges split across CTAs (swa_split.cuh):
+// schedule, attention over the schedule's list, merge of the split units.
+template <int D, bool SINK>
+int launch_chunk_split(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                       const CUtensorMap &tkr, const CUtensorMap &tvr, const CUtensorMap *tks,
+                       const CUtensorMap *tvs, swa::Fwd2Params p, void *workspace,
+                       cudaStream_t st) {
+  const int64_t units = fwd_units(p);
+  if (units > 0x7FFFFFFF) return SWA_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(units);
+  int P = 0;
+  if (sm_count(&P)) return SWA_ERR_CUDA;
+  int *ws = static_cast<int *>(workspace);
+  p.items = reinterpret_cast<const int4 *>(ws + swa::SplitLayout::kHeaderInts);
+  p.ws_ml = reinterpret_cast<float *>(ws) + swa::SplitLayout::ml_offset(units, P);
+  p.ws_o = reinterpret_cast<float *>(ws) + swa::SplitLayout::o_offset(units, P);
+  swa::chunk_split_schedule_kernel<D><<<1, swa::kSplitThreads, 0, st>>>(p, P, ws);
+  if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+  int e = launch_fwd<D, 1, SINK>(tq, tk, tv, tkr, tvr, p, st, tks, tvs, true);
+  if (e) return e;
+  swa::chunk_split_merge_kernel<D>
+      <<<dim3(P, 2, swa::kQT / swa::kMergeRowsPerCta), 32 * swa::kMergeRowsPerCta, 0, st>>>(p, P,
+                                                                                        ws);
+  return check_launch();
+}
 
 }  // namespace
 
@@ -351,7 +390,7 @@ int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring
                const int64_t *q_start, const int64_t *chunk_len, void *out, float *lse, int B,
                int H, int Hkv, int64_t Tq, int d, int64_t W, float scale, int update_ring,
                void *stream, const void *k_sink = nullptr, const void *v_sink = nullptr,
-               int n_sink = 0) {
+               int n_sink = 0, void *workspace = nullptr, size_t workspace_bytes = 0) {
   int e = common_checks(B, H, Hkv, d, W, scale);
   if (e) return e;
   if (!q || !k_new || !v_new || !k_ring || !v_ring || !q_start || !out) return SWA_ERR_INVALID_ARG;
@@ -390,12 +429,24 @@ int chunk_ring(const void *q, const void *k_new, const void *v_new, void *k_ring
   p.nqt = static_cast<int>((Tq + kBQ - 1) / kBQ);
   p.n_ring_tiles = static_cast<int>((W + kBK - 1) / kBK);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n_sink > 0)
+  if (workspace) {
+    if (workspace_bytes < swa_chunk_split_workspace_bytes(B, H, Hkv, Tq, d, W) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return SWA_ERR_WORKSPACE;
+    const CUtensorMap *ps = n_sink > 0 ? &tks : &tk, *pv = n_sink > 0 ? &tvs : &tv;
+    if (n_sink > 0)
+      e = d == 128 ? launch_chunk_split<128, true>(tq, tk, tv, tkr, tvr, ps, pv, p, workspace, st)
+                   : launch_chunk_split<64, true>(tq, tk, tv, tkr, tvr, ps, pv, p, workspace, st);
+    else
+      e = d == 128 ? launch_chunk_split<128, false>(tq, tk, tv, tkr, tvr, ps, pv, p, workspace, st)
+                   : launch_chunk_split<64, false>(tq, tk, tv, tkr, tvr, ps, pv, p, workspace, st);
+  } else if (n_sink > 0) {
     e = d == 128 ? launch_fwd<128, 1, true>(tq, tk, tv, tkr, tvr, p, st, &tks, &tvs)
                  : launch_fwd<64, 1, true>(tq, tk, tv, tkr, tvr, p, st, &tks, &tvs);
-  else
+  } else {
     e = d == 128 ? launch_fwd<128, 1>(tq, tk, tv, tkr, tvr, p, st)
                  : launch_fwd<64, 1>(tq, tk, tv, tkr, tvr, p, st);
+  }
   if (e || !update_ring) return e;
   return ring_write(k_new, v_new, k_ring, v_ring, q_start, chunk_len, B, Hkv, Tq, d, W, stream);
 }
@@ -417,6 +468,32 @@ int swa_attn_chunk_ring_sink(const void *q, const void *k_new, const void *v_new
   if (n_sink < 1) return SWA_ERR_INVALID_ARG;
   return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, nullptr, out, lse, B, H, Hkv, Tq, d,
                     W, scale, update_ring, stream, k_sink, v_sink, n_sink);
+}
+
+size_t swa_chunk_split_workspace_bytes(int B, int H, int Hkv, int64_t Tq, int d, int64_t W) {
+  if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Tq < 1 || W < 1 || (d != 64 && d != 128))
+    return 0;
+  swa::Fwd2Params p;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.nqt = static_cast<int>((Tq + kBQ - 1) / kBQ);
+  int P = 0;
+  if (sm_count(&P)) return 0;
+  return static_cast<size_t>(swa::SplitLayout::bytes(fwd_units(p), P, d));
+}
+
+int swa_attn_chunk_ring_split(const void *q, const void *k_new, const void *v_new, void *k_ring,
+                              void *v_ring, const void *k_sink, const void *v_sink, int n_sink,
+                              const int64_t *q_start, const int64_t *chunk_len, void *out,
+                              float *lse, int B, int H, int Hkv, int64_t Tq, int d, int64_t W,
+                              float scale, int update_ring, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+  if (!workspace) return SWA_ERR_WORKSPACE;
+  return chunk_ring(q, k_new, v_new, k_ring, v_ring, q_start, chunk_len, out, lse, B, H, Hkv, Tq,
+                    d, W, scale, update_ring, stream, k_sink, v_sink, n_sink, workspace,
+                    workspace_bytes);
 }
 
 int swa_attn_chunk_ring_ragged(const void *q, const void *k_new, const void *v_new,

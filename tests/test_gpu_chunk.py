@@ -319,3 +319,124 @@ def test_chunk_sink_workload_sampled_rows(swa):
     ref = oracle.swa_chunk_sink(q, kn, vn, rk, rv, sk, sv, qs, w.W, w.scale, rows=rows)
     got = to_f64(out)[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_close_bf16out(got, ref, what="chunk_ring_sink workload")
+
+
+# ---------------------------------------------------------------------------------------------
+# swa_attn_chunk_ring_split: the same chunk calls with a workspace, where the units of the
+# last round are cut into key-range parts across the SMs and merged.  Small batches have
+# few units, so here nearly every unit is split; the results must match the oracle as
+# the unsplit calls do, with padding rows and the ring update unchanged in meaning.
+
+def _run_split(swa, q, kn, vn, rk, rv, qs, scale, lens=None, sk=None, sv=None, update=False,
+               fill=7.0):
+    tq, tkn, tvn, trk, trv = (to_dev(x) for x in (q, kn, vn, rk, rv))
+    tqs = torch.tensor(qs, dtype=torch.int64, device="cuda")
+    tl = None if lens is None else torch.tensor(lens, dtype=torch.int64, device="cuda")
+    out = torch.full_like(tq, fill)
+    lse = torch.full(tq.shape[:3], fill, dtype=torch.float32, device="cuda")
+    swa.swa_attn_chunk_ring_split(tq, tkn, tvn, trk, trv, tqs, scale, chunk_len=tl,
+                                  k_sink=None if sk is None else to_dev(sk),
+                                  v_sink=None if sv is None else to_dev(sv), update_ring=update,
+                                  out=out, lse=lse, return_lse=True)
+    assert swa.swa_get_device_status() == 0
+    return out, lse, trk, trv
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,d,W,starts,lens", [
+    (4, 4, 2, 300, 128, 256, [512, 40, 0, 700], [300, 1, 129, 0]),
+    (3, 6, 2, 256, 64, 128, [1000, 3, 129], [200, 256, 65]),
+    (3, 8, 2, 384, 128, 512, [12288 + 37, 0, 511], [127, 128, 383]),
+    (2, 8, 2, 512, 128, 4096, [12288, 9000], [512, 512]),       # every chunk full
+])
+def test_split_ragged_chunks_per_sequence(swa, B, H, Hkv, Tq, d, W, starts, lens):
+    seed = 1900 + Tq + W
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    scale = 1.0 / math.sqrt(d)
+    out, lse, trk, trv = _run_split(swa, q, kn, vn, rk, rv, starts, scale, lens=lens,
+                                    update=True)
+    got, got_lse = to_f64(out), to_f64(lse)
+    erk, erv = rk.copy(), rv.copy()
+    for b, (qs, n) in enumerate(zip(starts, lens)):
+        assert np.all(got[b, :, n:] == 7.0)
+        assert np.all(got_lse[b, :, n:] == 7.0)
+        if n == 0:
+            continue
+        sl = (slice(b, b + 1), slice(None), slice(0, n))
+        ref, ref_lse = oracle.swa_chunk(q[sl], kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [qs], W,
+                                        scale, with_lse=True)
+        assert_close(got[b:b + 1, :, :n], ref, what=f"split chunk b={b} len={n}")
+        assert np.max(np.abs(got_lse[b:b + 1, :, :n] - ref_lse)) < 1e-3
+        k1, v1 = oracle.ring_update(kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [qs], W)
+        erk[b:b + 1], erv[b:b + 1] = k1, v1
+    assert np.array_equal(to_host_bits(trk), erk)
+    assert np.array_equal(to_host_bits(trv), erv)
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,d,W,S,starts", [
+    (2, 8, 2, 200, 128, 256, 4, [5000 + 77, 300]),
+    (3, 6, 2, 130, 64, 100, 16, [1000, 77, 3]),
+])
+def test_split_chunk_with_sinks(swa, B, H, Hkv, Tq, d, W, S, starts):
+    from tests._util import assert_close_bf16out
+
+    seed = 2100 + Tq + W + S
+    q = si.normal_bf16(seed, si.STREAM["q"], (B, H, Tq, d))
+    kn = si.normal_bf16(seed, si.STREAM["k_new"], (B, Hkv, Tq, d))
+    vn = si.normal_bf16(seed, si.STREAM["v_new"], (B, Hkv, Tq, d))
+    rk, rv = _ring_from_history(seed, B, Hkv, W, d, starts)
+    sk = si.normal_bf16(seed, si.STREAM["k_sink"], (B, Hkv, S, d))
+    sv = si.normal_bf16(seed, si.STREAM["v_sink"], (B, Hkv, S, d))
+    for b, qs in enumerate(starts):
+        for j in range(qs, min(S, qs + Tq)):
+            sk[b, :, j] = kn[b, :, j - qs]
+            sv[b, :, j] = vn[b, :, j - qs]
+    scale = 1.0 / math.sqrt(d)
+    out, lse, _, _ = _run_split(swa, q, kn, vn, rk, rv, starts, scale, sk=sk, sv=sv)
+    ref, ref_lse = oracle.swa_chunk_sink(q, kn, vn, rk, rv, sk, sv, starts, W, scale,
+                                         with_lse=True)
+    assert_close_bf16out(to_f64(out), ref, what="split chunk with sinks")
+    assert np.max(np.abs(to_f64(lse) - ref_lse)) < 1e-3
+
+
+def test_split_ragged_workload_every_valid_row(swa):
+    """The benchmarked ragged batch (1..512 valid rows per sequence) through the split call:
+    every valid output row against the oracle, padding untouched."""
+    from swa_inputs.workloads import seq_lens
+
+    w = WORKLOADS["chunk_ring_ragged"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    lens = [int(n) for n in seq_lens(w)]
+    out, _, _, _ = _run_split(swa, q, kn, vn, rk, rv, list(qs), w.scale, lens=lens)
+    got = to_f64(out)
+    for b, n in enumerate(lens):
+        sl = (slice(b, b + 1), slice(None), slice(0, n))
+        ref = oracle.swa_chunk(q[sl], kn[sl], vn[sl], rk[b:b + 1], rv[b:b + 1], [int(qs[b])],
+                               w.W, w.scale)
+        assert_close(got[b:b + 1, :, :n], ref, what=f"split ragged workload b={b}")
+        assert np.all(got[b, :, n:] == 7.0)
+
+
+def test_split_workload_matches_unsplit_call(swa):
+    """The chunk-ring workload through both calls: within the tolerance of each other
+    (the split changes only the summation order of the units it cuts)."""
+    w = WORKLOADS["chunk_ring"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    a = to_f64(_run(swa, q, kn, vn, rk, rv, list(qs), w.scale)[0])
+    b = to_f64(_run_split(swa, q, kn, vn, rk, rv, list(qs), w.scale)[0])
+    assert_close(b, a, what="split vs unsplit")
+
+
+def test_split_rejects_small_workspace(swa):
+    from sliding_window_sparse_b200._native import SwaError
+
+    B, H, Hkv, Tq, d, W = 1, 2, 2, 16, 64, 32
+    z = torch.zeros((B, H, Tq, d), dtype=torch.bfloat16, device="cuda")
+    zk = torch.zeros((B, Hkv, Tq, d), dtype=torch.bfloat16, device="cuda")
+    rk = torch.zeros((B, Hkv, W, d), dtype=torch.bfloat16, device="cuda")
+    qs = torch.tensor([40], dtype=torch.int64, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(SwaError):
+        swa.swa_attn_chunk_ring_split(z, zk, zk, rk, rk.clone(), qs, 0.1, workspace=ws)

@@ -238,3 +238,23 @@ def test_ring_write_stays_in_ring(swa, offset):
     rk2, rv2 = rk0.clone(), rv0.clone()
     swa.swa_ring_write(kn, vn, rk2, rv2, starts)
     assert torch.equal(rk.t, rk2) and torch.equal(rv.t, rv2)
+
+
+@pytest.mark.parametrize("offset", [0, 256])
+def test_chunk_split_out_lse_workspace_and_ring(swa, offset):
+    """The split chunk call writes inside out, lse, the ring and its workspace only."""
+    B, H, Hkv, Tq, d, W = 3, 4, 2, 200, 128, 256
+    starts = torch.tensor([1000 + 37, 64, 300], dtype=torch.int64, device="cuda")
+    lens = torch.tensor([200, 1, 129], dtype=torch.int64, device="cuda")
+    q, kn, vn, rk0, rv0 = _chunk_inputs(29, B, H, Hkv, Tq, d, W)
+    need = swa.swa_chunk_split_workspace_bytes(B, H, Hkv, Tq, d, W)
+    ws = Guarded((need,), torch.uint8, offset, fill=torch.zeros(()))
+    out = Guarded((B, H, Tq, d), torch.bfloat16, offset, fill=torch.zeros(()))
+    lse = Guarded((B, H, Tq), torch.float32, offset, fill=torch.zeros(()))
+    rk = Guarded((B, Hkv, W, d), torch.bfloat16, offset, fill=rk0)
+    rv = Guarded((B, Hkv, W, d), torch.bfloat16, offset, fill=rv0)
+    swa.swa_attn_chunk_ring_split(q, kn, vn, rk.t, rv.t, starts, 0.1, chunk_len=lens,
+                                  update_ring=True, out=out.t, lse=lse.t, workspace=ws.t)
+    assert swa.swa_get_device_status() == 0
+    for g in (ws, out, lse, rk, rv):
+        assert g.margins_intact()
