@@ -63,6 +63,26 @@ def test_small_shapes_full_tensor(swa, B, H, Hkv, N, d, W):
     assert_close(to_f64(out), ref, what=f"B{B} H{H}/{Hkv} N{N} d{d} W{W}")
 
 
+@pytest.mark.parametrize("B,H,Hkv,N,d,W", [
+    (1, 6, 2, 700, 128, 200),    # G = 3
+    (2, 2, 2, 1000, 128, 1024),  # eight-tile window
+    (1, 2, 2, 1000, 128, 1025),  # one more key
+    (1, 3, 3, 500, 64, 300),     # H odd
+    (1, 6, 6, 333, 64, 77),      # d = 64, ragged tail
+    (3, 4, 4, 130, 128, 129),    # two query tiles, the second of two rows
+])
+def test_query_tile_pairs_for_odd_groups(swa, B, H, Hkv, N, d, W):
+    """With G = H / Hkv odd a unit is query tiles 2p and 2p + 1 of one head
+    (the key stream is the union of both windows); against the oracle, with
+    the log-sum-exp."""
+    q, k, v = _inputs(300 + N + W, B, H, Hkv, N, d)
+    scale = 1.0 / math.sqrt(d)
+    out, lse = _run(swa, q, k, v, W, scale, lse=True)
+    ref, ref_lse = oracle.swa_forward(q, k, v, W, scale, with_lse=True)
+    assert_close(to_f64(out), ref, what=f"B{B} H{H}/{Hkv} N{N} d{d} W{W}")
+    assert np.max(np.abs(to_f64(lse) - ref_lse)) < 1e-3
+
+
 def test_worked_example_zero_scores(swa):
     """M003 note section 05: zero scores, V = 1..8 -> 7 (W = 3) and 4.5 (full)."""
     N, d = 8, 64

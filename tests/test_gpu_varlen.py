@@ -119,6 +119,8 @@ def test_varlen_bad_offsets_set_device_status(swa):
     (2, 8, 2, 700, 128, 128, 4),    # sink tile ahead of the window
     (1, 4, 4, 300, 128, 200, 4),    # window reaches tile 0 for the later query tiles
     (2, 6, 2, 513, 64, 64, 1),      # query-tile pairs, one sink
+    (2, 3, 1, 513, 64, 64, 1),      # G = 3 with H odd, one sink
+    (1, 2, 2, 3000, 128, 1500, 4),  # query-tile pairs, a window of twelve key tiles
     (1, 8, 2, 256, 128, 1000, 4),   # window covers everything: sinks change nothing
 ])
 def test_fwd_sink_full_tensor(swa, B, H, Hkv, N, d, W, S):
