@@ -190,6 +190,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "fwd2_kernel": ("swa_fwd2.cuh", "swa_tile.cuh", "swa_epilogue.cuh", "sm100.cuh"),
     "decode_split_kernel": ("swa_decode.cuh", "sm100.cuh"),
+    "bwd_kernels": ("swa_bwd.cuh", "swa_epilogue.cuh", "sm100.cuh"),
 }
 
 
@@ -665,9 +666,9 @@ def run_native(args):
                               "roofline": {"bound": "tensor", "achieved": tf,
                                            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                            "frac": tf / peaks["bf16_tflops"],
-                                           "traffic": (profiled_traffic("fwd2_kernel", name)
-                                                       if "backward" not in pw.kind
-                                                       else None)}})
+                                           "traffic": profiled_traffic(
+                                               "bwd_kernels" if "backward" in pw.kind
+                                               else "fwd2_kernel", name)}})
             if (rank == 0 and world == 1 and not args.no_cpu_baseline
                     and name in CPU_BASELINE_PATHS):
                 entry["cpu_baseline"] = cpu_baseline(pw, host_inputs_of(pw, px),

@@ -233,12 +233,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // unit -> (b, h, t) and its sequence; 0: run it, 1: bad sequence offsets
   // (skip, flag), 2: the query tile lies past the sequence's end (skip).
   // Every role evaluates it identically, so they skip the same units.
+  // Query tiles from the last down; on the packed layout sequence by
+  // sequence (so the key tiles of the units in flight stay in L2), elsewhere
+  // across every (b, head) at once.
   auto unit = [&](int u, int &b, int &h, int &t, int64_t &a, int &len) -> int {
-    const int per_t = p.B * p.H;
-    t = p.nt - 1 - u / per_t;
-    const int bh = u % per_t;
-    b = bh / p.H;
-    h = bh % p.H;
+    if (MODE == 2) {
+      const int per_b = p.H * p.nt, r = u % per_b;
+      b = u / per_b;
+      t = p.nt - 1 - r / p.H;
+      h = r % p.H;
+    } else {
+      const int per_t = p.B * p.H;
+      t = p.nt - 1 - u / per_t;
+      const int bh = u % per_t;
+      b = bh / p.H;
+      h = bh % p.H;
+    }
     if (bwd_seq<MODE>(p, b, a, len)) return 1;
     return t * kBwdT >= len ? 2 : 0;
   };
@@ -612,13 +622,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // 0: run it, 1: bad sequence offsets (skip, flag), 2: the key tile lies past
   // the sequence's end (skip).  Key tile 0 of every (b, kv head) first, then
   // key tile 1, and so on: the heaviest units first (with sinks, key tile 0
-  // is read by every query tile of its sequence).
+  // is read by every query tile of its sequence).  On the packed layout the
+  // units run sequence by sequence and, within one, KV head by KV head, so
+  // the query tiles that the units in flight read stay in L2.
   auto unit = [&](int u, int &b, int &kvh, int &kt, int &t_hi, int64_t &a, int &len) -> int {
-    const int per_t = p.B * p.Hkv;
-    kt = u / per_t;
-    const int bk = u % per_t;
-    b = bk / p.Hkv;
-    kvh = bk % p.Hkv;
+    if (MODE == 2) {
+      const int per_b = p.Hkv * p.nt, r = u % per_b;
+      b = u / per_b;
+      kvh = r / p.nt;
+      kt = r % p.nt;
+    } else {
+      const int per_t = p.B * p.Hkv;
+      kt = u / per_t;
+      const int bk = u % per_t;
+      b = bk / p.Hkv;
+      kvh = bk % p.Hkv;
+    }
     if (bwd_seq<MODE>(p, b, a, len)) return 1;
     if (kt * kBwdT >= len) return 2;
     const int nt_s = (len + kBwdT - 1) / kBwdT;

@@ -124,14 +124,31 @@ struct Unit {
   bool has_b;
 };
 
+// Unit order: query tile t from the last down (heavy first).  Head pairs on
+// the linear and ring layouts run t-major over every (sequence, pair), so
+// the units in flight share their key tiles across all sequences.  On the
+// packed layout they run sequence-major (t-major within each sequence): the
+// windows of many sequences at once would not stay in L2, and a unit whose
+// query tile lies past its sequence's end is skipped at no cost.
+template <int MODE = 0>
 __device__ __forceinline__ Unit decode_unit(int u, const Fwd2Params &p) {
   Unit U;
   if (p.pair_heads) {
     const int half = p.G >> 1;
-    const int per_t = p.B * p.Hkv * half;
-    const int t = p.nqt - 1 - u / per_t;
-    const int r = u % per_t;
-    const int pair = r % half, bk = r / half;
+    int t, r, bk;
+    if (MODE == 2) {
+      const int per_t = p.Hkv * half, per_b = per_t * p.nqt;
+      const int rb = u % per_b;
+      t = p.nqt - 1 - rb / per_t;
+      r = rb % per_t;
+      bk = (u / per_b) * p.Hkv + r / half;
+    } else {
+      const int per_t = p.B * p.Hkv * half;
+      t = p.nqt - 1 - u / per_t;
+      r = u % per_t;
+      bk = r / half;
+    }
+    const int pair = r % half;
     U.b = bk / p.Hkv;
     U.kvh = bk % p.Hkv;
     U.h[0] = U.kvh * p.G + 2 * pair;
@@ -504,7 +521,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
       bool k_ahead = false;  // K of iteration kv_iter issued, its V not (abort between them)
       int u, part, parts, slot;
       for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
-        Unit U = decode_unit(u, p);
+        Unit U = decode_unit<MODE>(u, p);
         int64_t qs;
         int len;
         const int ust = unit_start(U, qs, len);
@@ -616,7 +633,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
       };
       int u, part, parts, slot;
       for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
-        Unit U = decode_unit(u, p);
+        Unit U = decode_unit<MODE>(u, p);
         int64_t qs;
         int len;
         if (unit_start(U, qs, len)) continue;
@@ -745,7 +762,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
     bool stop = false;  // a wait gave up (the whole warp): no more TMEM work or stores
     int u, part, parts, slot;
     for (int it = 0; item_of(it, u, part, parts, slot); ++it) {
-      Unit U = decode_unit(u, p);
+      Unit U = decode_unit<MODE>(u, p);
       int64_t qs;
       int len;
       if (unit_start(U, qs, len)) continue;
