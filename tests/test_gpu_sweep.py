@@ -3,9 +3,10 @@
 Each case draws B, the head layout (G = H / Hkv in {1, 2, 3, 4, 8}), d, the
 window (from 1 to past the sequence), lengths that are not multiples of the
 128-row tile, chunk starts on either side of the ring's wrap and sink counts,
-so that edge combinations no hand-picked case covers are exercised.  Outputs
-are compared with the bf16-output bound (the 1e-2 bar plus 2^-8 of each
-value), mean-abs 1e-3.
+so that edge combinations no hand-picked case covers are exercised.  Prefill
+and packed rows that average at least 16 keys are held to the plain bar
+(max-abs 1e-2, mean-abs 1e-3); rows of fewer keys, and the chunk and decode
+cases, to the bf16-output bound (the 1e-2 bar plus 2^-8 of each value).
 """
 
 import math
@@ -16,7 +17,7 @@ import torch
 
 import oracle
 import swa_inputs as si
-from tests._util import assert_close_bf16out, to_dev, to_f64
+from tests._util import assert_close_bf16out, assert_close_by_keys, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -60,7 +61,8 @@ def test_sweep_prefill(swa, case):
     for b in range(B):
         tm = lambda x: np.ascontiguousarray(x[b].transpose(1, 0, 2))
         ref = oracle.swa_varlen(tm(q), tm(k), tm(v), [0, N], W, scale, n_sink=S)
-        assert_close_bf16out(got[b].transpose(1, 0, 2), ref,
+        keys = np.minimum(np.arange(N) + 1, W)[:, None]  # [rows, 1]: per token, every head
+        assert_close_by_keys(got[b].transpose(1, 0, 2), ref, keys,
                              what=f"prefill B{B} H{H}/{Hkv} N{N} d{d} W{W} S{S}")
 
 
@@ -152,7 +154,9 @@ def test_sweep_varlen(swa, case):
                               scale, n_sink=S)
     assert swa.swa_get_device_status() == 0
     ref = oracle.swa_varlen(q, k, v, cu, W, scale, n_sink=S)
-    assert_close_bf16out(to_f64(out), ref, what=f"varlen lens{lens} H{H}/{Hkv} d{d} W{W} S{S}")
+    pos = np.concatenate([np.arange(n) for n in lens])  # position of each token in its sequence
+    keys = np.minimum(pos + 1, W)[:, None]
+    assert_close_by_keys(to_f64(out), ref, keys, what=f"varlen lens{lens} H{H}/{Hkv} d{d} W{W} S{S}")
 
 
 @pytest.mark.parametrize("case", range(16))
