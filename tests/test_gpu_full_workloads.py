@@ -1,5 +1,7 @@
 """Every output element of the Mistral-shaped prefill, the narrow-window prefill
-and the chunk-on-ring workload against the fp64 oracle.
+and the chunk-on-ring workload (and of their variants with 4 attention sinks)
+against the fp64 oracle; and, for the Mistral-shaped backward, every gradient
+element of one key/value head group at the full size.
 
 The tolerance is the one stated for these workloads: max-abs 1e-2 and mean-abs
 1e-3 over the whole tensor (bf16 inputs, fp32 accumulation, bf16 output), plus
@@ -13,7 +15,8 @@ import pytest
 import torch
 
 import oracle
-from swa_inputs.workloads import WORKLOADS, chunk_inputs, prefill_inputs
+import swa_inputs as si
+from swa_inputs.workloads import WORKLOADS, chunk_inputs, prefill_inputs, sink_inputs
 from tests._util import MAX_ABS, MEAN_ABS, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -90,3 +93,69 @@ def test_chunk_ring_workload_every_element(swa):
     stats.add(out.float().cpu().numpy().astype(np.float64), ref)
     assert stats.count == w.B * w.H * w.Tq * w.d
     stats.check("chunk_ring")
+
+
+def test_sink_prefill_workload_every_element(swa):
+    """Mistral-shaped prefill with 4 sinks (taxonomy page section 3.2): every element."""
+    w = WORKLOADS["mistral_prefill_sink"]
+    q, k, v = prefill_inputs(w)
+    out = swa.swa_attn_fwd(to_dev(q), to_dev(k), to_dev(v), w.W, w.scale, n_sink=w.n_sink)
+    assert swa.swa_get_device_status() == 0
+    torch.cuda.synchronize()
+    G = w.H // w.Hkv
+    tm = lambda x: np.ascontiguousarray(x[0].transpose(1, 0, 2))  # noqa: E731  [N, heads, d]
+    stats = ErrorStats()
+    for h0 in range(0, w.H, 2 * G):
+        h1 = h0 + 2 * G
+        ref = oracle.swa_varlen(tm(q[:, h0:h1]), tm(k[:, h0 // G:h1 // G]),
+                                tm(v[:, h0 // G:h1 // G]), [0, w.N], w.W, w.scale,
+                                n_sink=w.n_sink)
+        stats.add(_gpu_slice_f64(out, 0, h0, h1), ref.transpose(1, 0, 2))
+    assert stats.count == w.B * w.H * w.N * w.d
+    stats.check("mistral_prefill_sink")
+
+
+def test_chunk_ring_sink_workload_every_element(swa):
+    """Chunk of 512 on a full ring with 4 sink rows: every element."""
+    w = WORKLOADS["chunk_ring_sink"]
+    q, kn, vn, rk, rv, qs = chunk_inputs(w)
+    sk, sv = sink_inputs(w)
+    out = swa.swa_attn_chunk_ring(to_dev(q), to_dev(kn), to_dev(vn), to_dev(rk), to_dev(rv),
+                                  torch.tensor(qs, dtype=torch.int64, device="cuda"), w.scale,
+                                  k_sink=to_dev(sk), v_sink=to_dev(sv))
+    assert swa.swa_get_device_status() == 0
+    ref = oracle.swa_chunk_sink(q, kn, vn, rk, rv, sk, sv, qs, w.W, w.scale)
+    stats = ErrorStats()
+    stats.add(out.float().cpu().numpy().astype(np.float64), ref)
+    assert stats.count == w.B * w.H * w.Tq * w.d
+    stats.check("chunk_ring_sink")
+
+
+def test_mistral_backward_one_group_every_element(swa):
+    """The benchmarked backward (B1 H32 Hkv8 N8192 d128 W4096) at its full size: the
+    gradients of key/value head 0's group (dq of query heads 0..G-1, dk and dv of key
+    head 0) depend on that group alone, so the oracle differentiates the group's slice
+    and every element of those gradients is compared.  Bounds per gradient tensor as
+    in the backward tests: max-abs <= 8u max|ref|, mean-abs <= 2u mean|ref|, relative
+    RMS <= 1e-2 (u = 2^-8)."""
+    w = WORKLOADS["mistral_backward"]
+    q, k, v = prefill_inputs(w)
+    g = si.normal_bf16(w.seed, si.STREAM["extra"], q.shape)
+    tq, tk, tv, tg = to_dev(q), to_dev(k), to_dev(v), to_dev(g)
+    out, lse = swa.swa_attn_fwd(tq, tk, tv, w.W, w.scale, return_lse=True)
+    dq, dk, dv = swa.swa_attn_bwd(tq, tk, tv, out, tg, lse, w.W, w.scale)
+    assert swa.swa_get_device_status() == 0
+    G = w.H // w.Hkv
+    rq, rk, rv = oracle.swa_backward(np.ascontiguousarray(q[:, :G]), np.ascontiguousarray(k[:, :1]),
+                                     np.ascontiguousarray(v[:, :1]), np.ascontiguousarray(g[:, :G]),
+                                     w.W, w.scale)
+    u = 2.0 ** -8
+    for name, got, ref in (("dq", dq[:, :G], rq), ("dk", dk[:, :1], rk), ("dv", dv[:, :1], rv)):
+        got = got.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(got)), f"{name}: non-finite"
+        err = np.abs(got - ref)
+        mx, mn = float(err.max()), float(err.mean())
+        rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+        assert mx <= 8 * u * float(np.abs(ref).max()), f"{name}: max-abs {mx:.3e}"
+        assert mn <= 2 * u * float(np.abs(ref).mean()), f"{name}: mean-abs {mn:.3e}"
+        assert rel <= 1e-2, f"{name}: relative RMS {rel:.3e}"
