@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import swa_inputs as si
-from tests._util import assert_close_bf16out, to_dev, to_f64
+from tests._util import assert_close_bf16out, assert_close_by_keys, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -156,6 +156,27 @@ def test_varlen_workload_sampled_rows(swa):
     rows = np.array([(t, int(rng.integers(w.H))) for t in toks], dtype=np.int64)
     ref = oracle.swa_varlen(q, k, v, cu, w.W, w.scale, n_sink=w.n_sink, rows=rows)
     assert_close_bf16out(got[rows[:, 0], rows[:, 1]], ref, what="varlen workload")
+
+
+def test_varlen_workload_whole_sequences_every_element(swa):
+    """The benchmarked packed batch: every output element (all heads) and the LSE of
+    each sequence of at most 4096 tokens and of the longest one, in the call that
+    packs all sixteen."""
+    from swa_inputs.workloads import WORKLOADS, varlen_inputs
+
+    w = WORKLOADS["varlen_prefill"]
+    q, k, v, cu = varlen_inputs(w)
+    got, got_lse = _run(swa, q, k, v, cu, w.W, w.scale, w.n_sink)
+    lens = np.diff(cu)
+    short = [s for s in range(len(lens)) if lens[s] <= 4096]
+    assert short
+    for s in short + [int(np.argmax(lens))]:
+        a, e = int(cu[s]), int(cu[s + 1])
+        ref, ref_lse = oracle.swa_varlen(q[a:e], k[a:e], v[a:e], [0, e - a], w.W, w.scale,
+                                         n_sink=w.n_sink, with_lse=True)
+        keys = np.minimum(np.arange(e - a) + 1, w.W)[:, None]
+        assert_close_by_keys(got[a:e], ref, keys, what=f"varlen workload seq {s} ({e - a} tokens)")
+        assert np.max(np.abs(got_lse[:, a:e] - ref_lse.T)) < 1e-3  # kernel LSE is [H, total]
 
 
 def test_sink_prefill_workload_sampled_rows(swa):
