@@ -234,3 +234,34 @@ def test_varlen_backward_workload_sampled(swa):
                                          w.W, w.scale, n_sink=w.n_sink)
         for name, x, y in zip(("dq", "dk", "dv"), (dq[a:e], dk[a:e], dv[a:e]), ref):
             _check(f"{name} seq {s} ({e - a} tokens)", to_f64(x), y)
+
+
+def test_varlen_backward_workload_long_sequence_one_group(swa):
+    """The benchmarked packed batch with sinks: every gradient element of its shortest
+    sequence longer than W + 1024 (5284 tokens: a thousand rows whose window no longer
+    reaches the 4 sinks) for key/value head 0's group (dq of its query heads, dk and dv
+    of the key head), which depend on that group and that sequence alone."""
+    from swa_inputs.workloads import WORKLOADS, seq_lens, varlen_inputs
+
+    w = WORKLOADS["varlen_backward"]
+    q, k, v, cu = varlen_inputs(w)
+    g = si.normal_bf16(w.seed, si.STREAM["extra"], q.shape)
+    tq, tk, tv, tg = to_dev(q), to_dev(k), to_dev(v), to_dev(g)
+    tcu = torch.tensor(cu, dtype=torch.int64, device="cuda")
+    lens = seq_lens(w)
+    max_len = int(max(lens))
+    out, lse = swa.swa_attn_varlen(tq, tk, tv, tcu, max_len, w.W, w.scale, n_sink=w.n_sink,
+                                   return_lse=True)
+    dq, dk, dv = swa.swa_attn_varlen_bwd(tq, tk, tv, tcu, max_len, out, tg, lse, w.W, w.scale,
+                                         n_sink=w.n_sink)
+    assert swa.swa_get_device_status() == 0
+    longer = [i for i in range(len(lens)) if lens[i] > w.W + 1024]
+    s = min(longer, key=lambda i: lens[i])
+    a, e = int(cu[s]), int(cu[s + 1])
+    G = w.H // w.Hkv
+    sl = lambda x, n: np.ascontiguousarray(x[a:e, :n])  # noqa: E731
+    ref = oracle.swa_varlen_backward(sl(q, G), sl(k, 1), sl(v, 1), sl(g, G),
+                                     np.array([0, e - a]), w.W, w.scale, n_sink=w.n_sink)
+    for name, x, y in zip(("dq", "dk", "dv"),
+                          (dq[a:e, :G], dk[a:e, :1], dv[a:e, :1]), ref):
+        _check(f"{name} seq {s} ({e - a} tokens), group 0", to_f64(x), y)
