@@ -339,6 +339,8 @@ SWA_API size_t swa_chunk_split_workspace_bytes(int B, int H, int Hkv, int64_t Tq
  *   workspace: device scratch of at least swa_chunk_split_workspace_bytes(B,
  *      H, Hkv, Tq, d, W) bytes, 256-byte aligned, caller-owned; contents on
  *      entry are ignored (SWA_ERR_WORKSPACE if missing, small or unaligned).
+ *      The call's kernels write it until the merge ends, so two calls in
+ *      flight at once (on different streams) need workspaces of their own.
  * Other arguments, layouts, limits and the ring update as swa_attn_chunk_ring.
  * Three kernels on `stream` (schedule, attention, merge), then the ring
  * update when update_ring != 0.
