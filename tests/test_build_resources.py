@@ -84,3 +84,20 @@ def test_backward_kernels_fit_their_block(report):
     assert len(bwd) == 16          # 2 kernels x D in {64, 128} x layout {0, 2} x SINK
     for name, r in bwd.items():
         assert r.get("regs", 0) <= 255, (name, r)
+
+
+def test_ring_layout_forward_spills_stay_small(report):
+    """The ring-layout (chunk) instantiations carry the split call's item list and
+    part bookkeeping; their spills stay a few words (16-20 bytes when this was
+    written), far from the softmax's score row."""
+    fwd = _fwd2(report)
+    for key, r in fwd.items():
+        if key[1] == 1:
+            assert r.get("spill", 0) <= 32, (key, r)
+
+
+def test_split_chunk_kernels_are_built(report):
+    """The split chunk call's schedule and merge kernels exist for d = 64 and 128."""
+    for kern in ("chunk_split_schedule_kernel", "chunk_split_merge_kernel"):
+        found = [n for n in report if kern in n]
+        assert len(found) == 2, (kern, found)
