@@ -88,12 +88,12 @@ def test_backward_kernels_fit_their_block(report):
 
 def test_ring_layout_forward_spills_stay_small(report):
     """The ring-layout (chunk) instantiations carry the split call's item list and
-    part bookkeeping; their spills stay a few words (16-20 bytes when this was
-    written), far from the softmax's score row."""
+    part bookkeeping; their spills stay a few words (16-20 bytes of stores plus
+    as many of loads when this was written), far from the softmax's score row."""
     fwd = _fwd2(report)
     for key, r in fwd.items():
         if key[1] == 1:
-            assert r.get("spill", 0) <= 32, (key, r)
+            assert r.get("spill", 0) <= 64, (key, r)  # spill stores + spill loads
 
 
 def test_split_chunk_kernels_are_built(report):
